@@ -1,0 +1,200 @@
+/*
+ * li.h -- C ABI of libli, a B200 (sm_100a) LightningIndexer.
+ *
+ * The operation (mindspore.ops.lightning_indexer page, ".. math::"; CANN
+ * LightningIndexerV2 guide, "三步计算流程"; VllmQuantLightningIndexer README,
+ * "功能说明"): for every query token and every key it may see,
+ *
+ *     s(t) = sum_h W[h] * ReLU( [Scale_Q[h] * Scale_K[t] *] (q_h . k_t) )
+ *
+ * then the sparse_count keys with the largest s (ties: lower key index first)
+ * are returned as int32 indices, optionally with their fp32 scores.
+ *
+ * Conventions shared by every entry point:
+ *   - The caller owns all memory.  Every tensor pointer is a DEVICE pointer to
+ *     a contiguous tensor (PA key blocks may be strided, see key_block_stride),
+ *     16-byte aligned.  The library allocates nothing and never synchronises
+ *     the stream, except li_read_device_status, which says so.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Every launch is asynchronous on it.
+ *   - A return value other than LI_OK means that nothing was launched; the
+ *     reason is in li_last_error() (a thread-local string).
+ *   - Errors that only the device can see (an actual length beyond the tensor
+ *     or the declared bound, a block id outside the pool, a negative dequant
+ *     scale, a bounded wait that expired) never fault: the kernels clamp or
+ *     skip the access and OR a bit into the status word at the start of the
+ *     workspace.  Read it with li_read_device_status.
+ */
+#ifndef LI_H
+#define LI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LI_API __attribute__((visibility("default")))
+#else
+#define LI_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LI_OK = 0,
+    LI_ERR_NULL = 1,         /* a required pointer is NULL                        */
+    LI_ERR_SHAPE = 2,        /* a dimension or attribute is out of range          */
+    LI_ERR_DTYPE = 3,        /* dtype combination not allowed                     */
+    LI_ERR_LAYOUT = 4,       /* layout combination not allowed                    */
+    LI_ERR_UNSUPPORTED = 5,  /* allowed by the pages but not built here           */
+    LI_ERR_WORKSPACE = 6,    /* workspace missing, too small or misaligned        */
+    LI_ERR_CUDA = 7,         /* a CUDA runtime call failed                        */
+    LI_ERR_DEVICE = 8        /* li_read_device_status: the device flagged a problem */
+} li_status;
+
+typedef enum { LI_BF16 = 0, LI_FP16 = 1, LI_FP32 = 2, LI_FP8_E4M3 = 3, LI_INT8 = 4 } li_dtype;
+typedef enum { LI_BSND = 0, LI_TND = 1, LI_PA_BSND = 2 } li_layout;
+
+/* Bits of the device status word (li_read_device_status). */
+#define LI_DEV_BAD_QLEN      0x01  /* query length / prefix sum out of range (clamped)  */
+#define LI_DEV_BAD_KLEN      0x02  /* key length / prefix sum out of range (clamped)    */
+#define LI_DEV_BAD_BLOCK     0x04  /* block_table entry outside [0, num_blocks) (skipped) */
+#define LI_DEV_NEG_SCALE     0x08  /* negative dequant scale (the fold needs scales >= 0) */
+#define LI_DEV_TIMEOUT       0x10  /* a bounded pipeline wait expired                   */
+
+/*
+ * Op attributes and dimensions (mindspore page, "参数" / "关键字参数"; CANN
+ * guide, "约束说明"; README, "参数说明").
+ *   layout_q       LI_BSND: query [B,S1,N1,D], weights [B,S1,N1]
+ *                  LI_TND : query [T1,N1,D],   weights [T1,N1]
+ *   layout_k       LI_BSND: key [B,S2,N2,D]; LI_TND: key [T2,N2,D];
+ *                  LI_PA_BSND: key [num_blocks,block_size,N2,D] addressed via block_table.
+ *                  Without PA, layout_k must equal layout_q.
+ *   dtype_qk       LI_BF16 / LI_FP16 (li_indexer), LI_FP8_E4M3 (li_quant_indexer)
+ *   dtype_w        LI_BF16 / LI_FP16 / LI_FP32
+ *   dtype_scale    LI_FP32 (li_quant_indexer only)
+ *   N1             query heads, 1..64;  N2 key heads, must be 1
+ *   D              head dim: 128, or 64 for 16-bit q/k (the TileLang test shape)
+ *   num_blocks, block_size, max_blocks_per_seq
+ *                  PA pool geometry; block_size a multiple of 16 in [16, 1024]
+ *   key_block_stride  elements between consecutive PA blocks (0 = dense
+ *                  block_size*N2*D); lets axis 0 of the pool be non-contiguous
+ *   sparse_count   k, 1..2048
+ *   sparse_mode    0 = every key inside the actual length; 3 = right-down causal:
+ *                  key t is visible to query i of batch b iff t <= i + Sk_b - Sq_b
+ *   pre_tokens, next_tokens  reserved; must be INT64_MAX
+ *   return_value   1 = also write sparse_values (fp32)
+ *   max_seqlen_k   host-side upper bound on every actual key length (0 = S2 for
+ *                  BSND, T2 for TND, max_blocks_per_seq*block_size for PA).  It
+ *                  sizes the workspace; longer actual lengths are clamped and flagged.
+ */
+typedef struct {
+    int32_t layout_q, layout_k;
+    int32_t dtype_qk, dtype_w, dtype_scale;
+    int32_t B, S1, S2, T1, T2, N1, N2, D;
+    int32_t num_blocks, block_size, max_blocks_per_seq;
+    int64_t key_block_stride;
+    int32_t sparse_count, sparse_mode;
+    int64_t pre_tokens, next_tokens;
+    int32_t return_value;
+    int32_t max_seqlen_k;
+} li_params;
+
+/*
+ * Output shape (CANN guide, "输出 shape 的推导依据"; mindspore page, "返回").
+ * BSND query: sparse_indices is [B, S1, N2, k] (ndim 4); TND: [T1, N2, k]
+ * (ndim 3).  sparse_values has the same shape when return_value is set.
+ * out_dims must hold 4 entries.  Host only; validates params.
+ */
+LI_API li_status li_output_shape(const li_params *p, int64_t out_dims[4], int32_t *ndim);
+
+/* Bytes of device workspace that li_indexer / li_quant_indexer need for `p`
+ * (status word, scheduler tables and one fp32 score row per query).  Host only. */
+LI_API li_status li_workspace_size(const li_params *p, size_t *bytes);
+
+/*
+ * The indexer on 16-bit query/key (mindspore page, whole signature; CANN guide,
+ * "函数原型").
+ *   query, key, weights   device tensors in the layouts above
+ *   act_seq_q  int32 [B]: per-batch query lengths for BSND (NULL = S1 each), or
+ *              prefix sums without a leading 0 for TND (required)
+ *   act_seq_k  int32 [B]: per-batch key lengths for BSND (NULL = S2 each) and
+ *              PA (required), or prefix sums for TND (required)
+ *   block_table int32 [B, max_blocks_per_seq], PA only: physical block of each
+ *              logical key block
+ *   sparse_indices  int32 [rows, k] output; slots past min(k, visible) are -1
+ *   sparse_values   fp32 [rows, k] output (NULL iff return_value == 0); padding -inf
+ *   workspace       device buffer of li_workspace_size bytes, 256-byte aligned;
+ *                   it must not be shared by calls that may run concurrently
+ */
+LI_API li_status li_indexer(const li_params *p, const void *query, const void *key, const void *weights,
+                     const int32_t *act_seq_q, const int32_t *act_seq_k,
+                     const int32_t *block_table, int32_t *sparse_indices, float *sparse_values,
+                     void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * The quantised indexer (VllmQuantLightningIndexer README, "功能说明"):
+ * q/k are fp8 e4m3, and the per-token-head dequant scales multiply the dot
+ * product before the ReLU.
+ *   q_scale  fp32, same layout as weights ([B,S1,N1] or [T1,N1])
+ *   k_scale  fp32 per key token: [B,S2,N2], [T2,N2] or [num_blocks,block_size,N2]
+ * Scales must be >= 0 (then ReLU(sq*sk*x) = sq*sk*ReLU(x), which the kernel
+ * uses); a negative scale is flagged with LI_DEV_NEG_SCALE.  Other arguments
+ * as li_indexer.
+ */
+LI_API li_status li_quant_indexer(const li_params *p, const void *query, const void *key,
+                           const void *weights, const float *q_scale, const float *k_scale,
+                           const int32_t *act_seq_q, const int32_t *act_seq_k,
+                           const int32_t *block_table, int32_t *sparse_indices,
+                           float *sparse_values, void *workspace, size_t workspace_bytes,
+                           void *stream);
+
+/*
+ * The Top-k stage on its own (CANN guide, "三步计算流程" step 3, with the
+ * deterministic ordering of "确定性计算"): for each of `rows` fp32 score rows
+ * (row r starts at scores + r*ld and its first row_len[r] entries are the
+ * candidates; row_len NULL = ld for every row), write the k largest as
+ * (index, value) pairs ordered by value descending, ties by lower index; pad
+ * with -1 / -inf.  -0.0 counts as +0.0.  ld must be a multiple of 4.
+ * sparse_values may be NULL.  Needs no workspace.
+ */
+LI_API li_status li_topk(const float *scores, int64_t ld, const int32_t *row_len, int32_t rows,
+                  int32_t k, int32_t *sparse_indices, float *sparse_values, void *stream);
+
+/* Thread-local message describing the last non-OK status. */
+LI_API const char *li_last_error(void);
+
+/*
+ * SYNCHRONISING: copy the device status word of `workspace` to the host after
+ * everything queued on `stream` has finished.  *flags receives the LI_DEV_*
+ * bits of the last call that used this workspace.  Returns LI_ERR_DEVICE when
+ * any bit is set, LI_OK otherwise.
+ */
+LI_API li_status li_read_device_status(const void *workspace, void *stream, int32_t *flags);
+
+/*
+ * Self-test of the bounded wait used by every pipeline barrier: one thread
+ * waits on a shared-memory barrier that nothing will ever complete, gives up
+ * after timeout_ns nanoseconds and ORs LI_DEV_TIMEOUT into *status_word (a
+ * device int32).  Lets a test check that an expired wait reports an error and
+ * leaves the context usable, without faulting or hanging the GPU.
+ */
+LI_API li_status li_selftest_bounded_wait(int32_t *status_word, int64_t timeout_ns, void *stream);
+
+/*
+ * Per-stage timing: when `events` holds n >= 4 cudaEvent_t handles (passed as
+ * void*), every later li_indexer / li_quant_indexer call on this thread records
+ * events[0] before the scheduler, events[1] after it, events[2] after the score
+ * kernel and events[3] after the Top-k kernel, on the call's stream.  n = 0 or
+ * events = NULL turns it off.  The handles are borrowed, not owned.
+ */
+LI_API void li_set_profile_events(void *const *events, int32_t n);
+
+/* Number of kernels launched by the last successful call on this thread. */
+LI_API int32_t li_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LI_H */

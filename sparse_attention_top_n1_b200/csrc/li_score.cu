@@ -1,0 +1,484 @@
+// li_score.cu -- the fused score kernel: s(t) for every visible (query, key).
+//
+// Computes, per query token i and key t (mindspore.ops.lightning_indexer page,
+// ".. math::"; CANN LightningIndexerV2 guide, "三步计算流程"; for fp8 the
+// VllmQuantLightningIndexer README, "功能说明"):
+//
+//     s(i,t) = [Scale_K(t) *] sum_h [W(i,h) * Scale_Q(i,h)] * ReLU(q(i,h) . k(t))
+//
+// (for scales >= 0 this equals sum_h W * ReLU(Scale_Q * Scale_K * q.k), the
+// README's order) and stores it, for the keys the sparse mode leaves visible,
+// into one fp32 score row per query.  Per-head logits never leave the SM.
+//
+// Design (one persistent CTA per SM, warp-specialised):
+//   warp 0     TMA producer: loads the query block (all heads of up to
+//              256/N1P queries, K-major, 128-byte swizzle) once per block and
+//              streams 128-key tiles through a STAGES-deep ring; paged keys
+//              are gathered block by block through block_table.
+//   warp 1     allocates 512 TMEM columns and issues tcgen05.mma
+//              (M = 128 keys, N = queries*heads <= 256, K = D) into one of two
+//              fp32 TMEM accumulators, then commits to the ring / accumulator
+//              barriers.
+//   warps 2-9  epilogue: each thread owns one key (one TMEM lane), loads that
+//              lane's head columns with tcgen05.ld and reduces them in
+//              registers -- ReLU, multiply by the weight, sum over heads, scale
+//              -- then writes the score if the key is visible.
+// Work is a flat list of (query block, key tile) units written by the
+// device-side scheduler; each CTA takes a contiguous, equal share, so causal
+// triangles and ragged lengths are balanced over the SMs.
+#include <cstdint>
+#include <cuda_fp16.h>
+
+#include "li_internal.cuh"
+#include "ptx.cuh"
+
+namespace li {
+namespace {
+
+constexpr int kRowBytes = 128;                        // one swizzle row
+constexpr int kQRows = 256;
+
+template <int CHUNKS>
+struct Geometry {
+    static constexpr int STAGES = CHUNKS == 2 ? 4 : 6;
+    static constexpr int Q_BYTES = kQRows * kRowBytes * CHUNKS;
+    static constexpr int Q_CHUNK = kQRows * kRowBytes;
+    static constexpr int K_CHUNK = kTileKeys * kRowBytes;
+    static constexpr int K_BYTES = K_CHUNK * CHUNKS;
+    static constexpr int W_FLOATS = kEpiWarps * 128;
+    static constexpr int NBARS = 2 * STAGES + 7;
+    static constexpr size_t SMEM = 1024 + Q_BYTES + (size_t)STAGES * K_BYTES + W_FLOATS * 4 +
+                                   NBARS * 8 + 16;
+};
+
+// Walks the flat unit list: unit u -> (query block qb, key tile).
+struct Walker {
+    const BlockInfo *blocks;
+    int nblocks;
+    int qb, tile, ntiles;
+    __device__ void init(int u)
+    {
+        int lo = 0, hi = nblocks - 1;                  // last block with unit_start <= u
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (blocks[mid].unit_start <= u) lo = mid; else hi = mid - 1;
+        }
+        qb = lo;
+        tile = u - blocks[lo].unit_start;
+        ntiles = blocks[lo].ntiles;
+    }
+    __device__ void next()
+    {
+        if (++tile >= ntiles) {
+            tile = 0;
+            do {
+                ++qb;
+                ntiles = qb < nblocks ? blocks[qb].ntiles : 1;
+            } while (ntiles == 0);
+        }
+    }
+};
+
+__device__ __forceinline__ float load_weight(const void *w, int dtype, int64_t i)
+{
+    if (dtype == LI_FP32) return static_cast<const float *>(w)[i];
+    const unsigned short h = static_cast<const unsigned short *>(w)[i];
+    if (dtype == LI_BF16) return __uint_as_float((uint32_t)h << 16);
+    return __half2float(__ushort_as_half(h));
+}
+
+__device__ __forceinline__ void fail(PlanHeader *hdr, volatile int *abort_flag, int bit)
+{
+    atomicOr(&hdr->status, bit);
+    *abort_flag = 1;
+}
+
+template <int CHUNKS, int N1P, bool FP8>
+__global__ void __launch_bounds__(kScoreThreads, 1)
+    score_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+                 const ScoreArgs a)
+{
+    using G = Geometry<CHUNKS>;
+    constexpr int STAGES = G::STAGES;
+    constexpr int NQ = 256 / N1P;                 // queries per block
+    constexpr int QPW = 128 / N1P;                // queries per epilogue warp half
+    constexpr int NP = N1P >= 32 ? 4 : (N1P == 16 ? 2 : 1);   // partial sums per query
+    constexpr int INNER = FP8 ? 128 : 64;         // elements per 128-byte row chunk
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = smem;
+    uint8_t *sK = smem + G::Q_BYTES;
+    float *sW = reinterpret_cast<float *>(sK + STAGES * G::K_BYTES);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sW + G::W_FLOATS);
+    uint64_t *k_full = bars;
+    uint64_t *k_empty = bars + STAGES;
+    uint64_t *q_full = bars + 2 * STAGES;
+    uint64_t *q_empty = q_full + 1;
+    uint64_t *acc_full = q_full + 2;
+    uint64_t *acc_empty = q_full + 4;
+    uint64_t *drain = q_full + 6;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + G::NBARS);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+        }
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
+        for (int s = 0; s < kAccStages; ++s) {
+            mbar_init(&acc_full[s], 1);
+            mbar_init(&acc_empty[s], kEpiWarps);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    if (a.q_box_rows != kQRows) {
+        // per-query Q boxes leave the padded head rows untouched: zero them once
+        uint4 *q4 = reinterpret_cast<uint4 *>(sQ);
+        for (int j = tid; j < G::Q_BYTES / 16; j += kScoreThreads) q4[j] = make_uint4(0, 0, 0, 0);
+        fence_proxy_async_smem();
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, 2 * kAccCols);
+    if (tid == 0) {
+        tma_prefetch_desc(&qmap);
+        tma_prefetch_desc(&kmap);
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int total = a.hdr->total_units;
+    const int nblocks = a.hdr->total_blocks;
+    const int u_begin = (int)(((int64_t)total * blockIdx.x) / gridDim.x);
+    const int u_end = (int)(((int64_t)total * (blockIdx.x + 1)) / gridDim.x);
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0 && u_begin < u_end) {
+            Walker w{a.blocks, nblocks, 0, 0, 0};
+            w.init(u_begin);
+            int stage = 0, prev_qb = -1;
+            uint32_t phase = 0, qphase = 0;
+            uint32_t armed = 0, par = 0, q_armed = 0, q_par = 0;
+            BlockInfo blk{};
+            BatchInfo bi{};
+            for (int u = u_begin; u < u_end; ++u) {
+                if (w.qb != prev_qb) {
+                    blk = a.blocks[w.qb];
+                    bi = a.batches[blk.b];
+                    if (!mbar_wait_bounded(q_empty, qphase ^ 1u, abort_flag, a.timeout_ns)) {
+                        fail(a.hdr, abort_flag, LI_DEV_TIMEOUT);
+                        break;
+                    }
+                    const int qrow0 = bi.q_off + blk.i0;
+                    if (a.q_box_rows == kQRows) {
+                        mbar_arrive_expect_tx(q_full, CHUNKS * G::Q_CHUNK);
+                        for (int c = 0; c < CHUNKS; ++c)
+                            tma_load_2d(sQ + c * G::Q_CHUNK, &qmap, q_full, c * INNER, qrow0 * a.N1);
+                    } else {
+                        mbar_arrive_expect_tx(q_full, CHUNKS * NQ * a.N1 * kRowBytes);
+                        for (int qi = 0; qi < NQ; ++qi)
+                            for (int c = 0; c < CHUNKS; ++c)
+                                tma_load_2d(sQ + c * G::Q_CHUNK + qi * N1P * kRowBytes, &qmap,
+                                            q_full, c * INNER, (qrow0 + qi) * a.N1);
+                    }
+                    q_armed = 1;
+                    q_par = qphase;
+                    qphase ^= 1u;
+                    prev_qb = w.qb;
+                }
+                if (!mbar_wait_bounded(&k_empty[stage], phase ^ 1u, abort_flag, a.timeout_ns)) {
+                    fail(a.hdr, abort_flag, LI_DEV_TIMEOUT);
+                    break;
+                }
+                uint8_t *dst = sK + stage * G::K_BYTES;
+                const int t0 = w.tile * kTileKeys;
+                if (!a.is_pa) {
+                    mbar_arrive_expect_tx(&k_full[stage], G::K_BYTES);
+                    for (int c = 0; c < CHUNKS; ++c)
+                        tma_load_2d(dst + c * G::K_CHUNK, &kmap, &k_full[stage], c * INNER,
+                                    bi.k_off + t0);
+                } else {
+                    // gather the tile from the paged pool, g = pa_box_rows keys at a time
+                    const int g = a.pa_box_rows, nseg = kTileKeys / g;
+                    int blkid[8];
+                    int nvalid = 0;
+                    for (int s = 0; s < nseg; ++s) {
+                        const int t = t0 + s * g;
+                        blkid[s] = -1;
+                        if (t >= bi.Sk) continue;
+                        const int id = a.block_table[(int64_t)blk.b * a.max_blocks_per_seq +
+                                                     t / a.block_size];
+                        if (id < 0 || id >= a.num_blocks) {
+                            atomicOr(&a.hdr->status, LI_DEV_BAD_BLOCK);
+                            continue;
+                        }
+                        blkid[s] = id;
+                        ++nvalid;
+                    }
+                    mbar_arrive_expect_tx(&k_full[stage], nvalid * g * kRowBytes * CHUNKS);
+                    for (int s = 0; s < nseg; ++s) {
+                        if (blkid[s] < 0) continue;
+                        const int t = t0 + s * g;
+                        for (int c = 0; c < CHUNKS; ++c)
+                            tma_load_3d(dst + c * G::K_CHUNK + s * g * kRowBytes, &kmap,
+                                        &k_full[stage], c * INNER, t % a.block_size, blkid[s]);
+                    }
+                }
+                armed |= 1u << stage;
+                par = (par & ~(1u << stage)) | (phase << stage);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+                w.next();
+            }
+            if (*abort_flag) {
+                // let every copy still in flight land before the CTA exits
+                for (int s = 0; s < STAGES; ++s)
+                    if (armed & (1u << s))
+                        mbar_wait_bounded(&k_full[s], (par >> s) & 1u, nullptr, a.timeout_ns);
+                if (q_armed) mbar_wait_bounded(q_full, q_par, nullptr, a.timeout_ns);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && u_begin < u_end) {
+            Walker w{a.blocks, nblocks, 0, 0, 0};
+            w.init(u_begin);
+            int stage = 0, acc = 0, prev_qb = -1;
+            uint32_t phase = 0, acc_phase = 0, qphase = 0, idesc = 0;
+            bool issued = false;
+            const uint32_t sQ_addr = smem_u32(sQ), sK_addr = smem_u32(sK);
+            for (int u = u_begin; u < u_end; ++u) {
+                if (w.qb != prev_qb) {
+                    const BlockInfo blk = a.blocks[w.qb];
+                    const BatchInfo bi = a.batches[blk.b];
+                    int nrows = bi.Sq - blk.i0;
+                    nrows = nrows > NQ ? NQ : nrows;
+                    int n = ((nrows * N1P + 15) / 16) * 16;
+                    n = n < 16 ? 16 : (n > kAccCols ? kAccCols : n);
+                    idesc = a.idesc_base | ((uint32_t)(n >> 3) << 17);
+                    if (!mbar_wait_bounded(q_full, qphase, abort_flag, a.timeout_ns)) {
+                        fail(a.hdr, abort_flag, LI_DEV_TIMEOUT);
+                        break;
+                    }
+                    qphase ^= 1u;
+                    prev_qb = w.qb;
+                }
+                if (!mbar_wait_bounded(&k_full[stage], phase, abort_flag, a.timeout_ns) ||
+                    !mbar_wait_bounded(&acc_empty[acc], acc_phase ^ 1u, abort_flag, a.timeout_ns)) {
+                    fail(a.hdr, abort_flag, LI_DEV_TIMEOUT);
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
+                const uint32_t k_addr = sK_addr + stage * G::K_BYTES;
+#pragma unroll
+                for (int c = 0; c < CHUNKS; ++c) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t ad = smem_desc_sw128(k_addr + c * G::K_CHUNK + kk * 32);
+                        const uint64_t bd = smem_desc_sw128(sQ_addr + c * G::Q_CHUNK + kk * 32);
+                        if (FP8)
+                            mma_f8(d_tmem, ad, bd, idesc, (c | kk) != 0);
+                        else
+                            mma_f16(d_tmem, ad, bd, idesc, (c | kk) != 0);
+                    }
+                }
+                issued = true;
+                mma_commit(&k_empty[stage]);
+                mma_commit(&acc_full[acc]);
+                if (w.tile + 1 == w.ntiles) mma_commit(q_empty);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+                if (++acc == kAccStages) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+                w.next();
+            }
+            if (issued) {
+                // every MMA of this CTA has finished before TMEM is released
+                mma_commit(drain);
+                mbar_wait_bounded(drain, 0, nullptr, a.timeout_ns);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int ew = warp - 2;                   // 0..7
+        const int quarter = warp & 3;              // TMEM lanes this warp may access
+        const int half = ew >> 2;                  // which 128 of the 256 columns
+        const int lrow = quarter * 32 + lane;      // key row within the tile
+        float *myW = sW + ew * 128;
+        if (u_begin < u_end) {
+            Walker w{a.blocks, nblocks, 0, 0, 0};
+            w.init(u_begin);
+            int acc = 0, prev_qb = -1, nchunks = 0;
+            uint32_t acc_phase = 0;
+            BlockInfo blk{};
+            BatchInfo bi{};
+            for (int u = u_begin; u < u_end; ++u) {
+                if (w.qb != prev_qb) {
+                    blk = a.blocks[w.qb];
+                    bi = a.batches[blk.b];
+                    int nrows = bi.Sq - blk.i0;
+                    nrows = nrows > NQ ? NQ : nrows;
+                    int mine = nrows - half * QPW;     // valid queries of this half
+                    mine = mine < 0 ? 0 : (mine > QPW ? QPW : mine);
+                    nchunks = (mine * N1P + 31) / 32;
+                    __syncwarp();
+                    for (int j = lane; j < 128; j += 32) {
+                        const int col = half * 128 + j;
+                        const int q = col / N1P, h = col % N1P;
+                        const int i = blk.i0 + q;
+                        float wv = 0.f;
+                        if (h < a.N1 && i < bi.Sq) {
+                            const int64_t r = (int64_t)(bi.q_off + i) * a.N1 + h;
+                            wv = load_weight(a.weights, a.dtype_w, r);
+                            if (a.quant) {
+                                const float sq = a.q_scale[r];
+                                if (sq < 0.f) atomicOr(&a.hdr->status, LI_DEV_NEG_SCALE);
+                                wv *= sq;
+                            }
+                        }
+                        myW[j] = wv;
+                    }
+                    __syncwarp();
+                    prev_qb = w.qb;
+                }
+                if (!mbar_wait_bounded(&acc_full[acc], acc_phase, abort_flag, a.timeout_ns)) {
+                    fail(a.hdr, abort_flag, LI_DEV_TIMEOUT);
+                    break;
+                }
+                tc_fence_after_sync();
+                const int t = w.tile * kTileKeys + lrow;
+                float ks = 1.f;
+                if (a.quant && t < bi.Sk) {
+                    int64_t kr = -1;
+                    if (!a.is_pa) {
+                        kr = (int64_t)bi.k_off + t;
+                    } else {
+                        const int id = a.block_table[(int64_t)blk.b * a.max_blocks_per_seq +
+                                                     t / a.block_size];
+                        if (id >= 0 && id < a.num_blocks)
+                            kr = (int64_t)id * a.block_size + t % a.block_size;
+                    }
+                    if (kr >= 0) {
+                        ks = a.k_scale[kr];
+                        if (ks < 0.f) atomicOr(&a.hdr->status, LI_DEV_NEG_SCALE);
+                    }
+                }
+                float part[QPW][NP];
+#pragma unroll
+                for (int q = 0; q < QPW; ++q)
+#pragma unroll
+                    for (int p = 0; p < NP; ++p) part[q][p] = 0.f;
+                const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16) +
+                                      (uint32_t)(acc * kAccCols + half * 128);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    if (c < nchunks) {
+                        float v[32];
+                        tmem_ld32(trow + c * 32, v);
+                        tmem_ld_wait();
+                        const float4 *w4 = reinterpret_cast<const float4 *>(myW + c * 32);
+#pragma unroll
+                        for (int j4 = 0; j4 < 8; ++j4) {
+                            const float4 ww = w4[j4];
+                            const float wj[4] = {ww.x, ww.y, ww.z, ww.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int j = j4 * 4 + e;
+                                const int q = (c * 32 + j) / N1P;
+                                part[q][j % NP] = fmaf(wj[e], fmaxf(v[j], 0.f), part[q][j % NP]);
+                            }
+                        }
+                    }
+                }
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[acc]);
+                if (++acc == kAccStages) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+                // visible keys only: t < nvis(i); the row keeps its visible prefix
+#pragma unroll
+                for (int q = 0; q < QPW; ++q) {
+                    const int i = blk.i0 + half * QPW + q;
+                    if (half * QPW + q < NQ && i < bi.Sq) {
+                        int nv = bi.Sk;
+                        if (a.mode == 3) {
+                            const int lim = i + 1 + bi.Sk - bi.Sq;
+                            nv = lim < 0 ? 0 : (lim < bi.Sk ? lim : bi.Sk);
+                        }
+                        if (t < nv) {
+                            float s = 0.f;
+#pragma unroll
+                            for (int p = 0; p < NP; ++p) s += part[q][p];
+                            a.scores[(int64_t)(bi.row0 + i) * a.ld + t] = s * ks;
+                        }
+                    }
+                }
+                w.next();
+            }
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    if (warp == 1) tmem_dealloc(tmem_base, 2 * kAccCols);
+}
+
+template <int CHUNKS, int N1P, bool FP8>
+cudaError_t launch_one(const ScoreArgs &a, const CUtensorMap &qmap, const CUtensorMap &kmap,
+                       int grid, cudaStream_t s)
+{
+    auto kern = score_kernel<CHUNKS, N1P, FP8>;
+    const size_t smem = Geometry<CHUNKS>::SMEM;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kScoreThreads, smem, s>>>(qmap, kmap, a);
+    return cudaGetLastError();
+}
+
+template <int CHUNKS, bool FP8>
+cudaError_t launch_n1p(const ScoreArgs &a, int n1p, const CUtensorMap &qmap,
+                       const CUtensorMap &kmap, int grid, cudaStream_t s)
+{
+    switch (n1p) {
+    case 8: return launch_one<CHUNKS, 8, FP8>(a, qmap, kmap, grid, s);
+    case 16: return launch_one<CHUNKS, 16, FP8>(a, qmap, kmap, grid, s);
+    case 32: return launch_one<CHUNKS, 32, FP8>(a, qmap, kmap, grid, s);
+    case 64: return launch_one<CHUNKS, 64, FP8>(a, qmap, kmap, grid, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+size_t score_smem_bytes(int chunks) { return chunks == 2 ? Geometry<2>::SMEM : Geometry<1>::SMEM; }
+int score_stages(int chunks) { return chunks == 2 ? Geometry<2>::STAGES : Geometry<1>::STAGES; }
+
+cudaError_t launch_score(const ScoreArgs &a, const Tiling &t, const CUtensorMap &qmap,
+                         const CUtensorMap &kmap, int fp8, int grid, cudaStream_t s)
+{
+    if (fp8) return t.chunks == 1 ? launch_n1p<1, true>(a, t.n1p, qmap, kmap, grid, s)
+                                  : cudaErrorInvalidValue;
+    return t.chunks == 2 ? launch_n1p<2, false>(a, t.n1p, qmap, kmap, grid, s)
+                         : launch_n1p<1, false>(a, t.n1p, qmap, kmap, grid, s);
+}
+
+}  // namespace li

@@ -1,0 +1,380 @@
+// li_topk.cu -- per-row Top-k over fp32 score rows.
+//
+// Step 3 of the CANN LightningIndexerV2 guide ("三步计算流程": keep the k
+// best positions) with the deterministic order of its "确定性计算" section,
+// read as: value descending, ties by lower key index; slots past the number
+// of candidates hold -1 / -inf ("通用约束").
+//
+// One CTA of 512 threads per row:
+//   1. Radix select.  Scores are mapped to order-preserving uint32 keys
+//      (-0.0 is first folded into +0.0).  Three histogram passes over the row
+//      (11, 11 and 10 bits, most significant first) find the exact key T of
+//      the k-th largest element and how many of the k must be taken from the
+//      elements equal to T.
+//   2. Compaction in index order: every key > T, plus the lowest-index keys
+//      == T, written to a buffer in ascending index order.
+//   3. A stable LSB radix sort of the selected keys by descending value (4
+//      passes of 8 bits; a pass whose digit is the same for every selected
+//      key is skipped).  Stability keeps equal values in index order.
+//   4. Write indices and values, pad with -1 / -inf.
+// Rows of up to `cap` elements are cached in shared memory; longer rows are
+// streamed from global memory (L2) on every pass.
+#include <cstdint>
+
+#include "li_internal.cuh"
+
+namespace li {
+namespace {
+
+constexpr int kWarps = kTopkThreads / 32;
+constexpr int kSortMaxRounds = 4;     // kmax <= 2048: 128 elements per warp
+
+__device__ __forceinline__ uint32_t to_key(float f)
+{
+    f = f + 0.0f;                                  // -0.0 -> +0.0
+    uint32_t b = __float_as_uint(f);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ float from_key(uint32_t u)
+{
+    uint32_t b = (u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u;
+    return __uint_as_float(b);
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt()
+{
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// Exclusive scan of one value per thread over the whole CTA; also returns the
+// total.  `tmp` holds kWarps + 1 ints.  Contains __syncthreads.
+template <typename T>
+__device__ __forceinline__ T block_exclusive_scan(T v, T *tmp, T &total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    T x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        T y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) tmp[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        T w = lane < kWarps ? tmp[lane] : T(0);
+        T s = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            T y = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o) s += y;
+        }
+        if (lane < kWarps) tmp[lane] = s - w;          // exclusive warp offsets
+        if (lane == kWarps - 1) tmp[kWarps] = s;       // total
+    }
+    __syncthreads();
+    T r = tmp[warp] + x - v;
+    total = tmp[kWarps];
+    __syncthreads();
+    return r;
+}
+
+struct RowSrc {
+    const float *g;       // row in global memory
+    const uint32_t *c;    // row cached as keys in shared memory (or null)
+    int n;
+    __device__ __forceinline__ uint4 load4(int j4) const
+    {
+        // keys j4*4 .. j4*4+3; entries >= n are never used by callers
+        if (c) return reinterpret_cast<const uint4 *>(c)[j4];
+        float4 v = reinterpret_cast<const float4 *>(g)[j4];
+        return make_uint4(to_key(v.x), to_key(v.y), to_key(v.z), to_key(v.w));
+    }
+};
+
+__global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a)
+{
+    extern __shared__ __align__(16) uint8_t smem[];
+    __shared__ uint32_t s_tmp32[kWarps + 1];
+    __shared__ uint64_t s_tmp64[kWarps + 1];
+    __shared__ uint32_t s_digit, s_above, s_or, s_and;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int row = blockIdx.x;
+    const int k = a.k;
+
+    // --- which elements of which row
+    int n = 0;
+    if (a.standalone) {
+        n = a.row_len ? a.row_len[row] : (int)a.ld;
+        n = n < 0 ? 0 : (n > a.ld ? (int)a.ld : n);
+    } else {
+        int b = -1, i = 0;
+        if (a.layout_q == LI_BSND) {
+            b = row / a.S1;
+            i = row % a.S1;
+        } else {
+            int lo = 0, hi = a.B - 1;               // last batch with q_off <= row
+            while (lo < hi) {
+                int mid = (lo + hi + 1) >> 1;
+                if (a.batches[mid].q_off <= row) lo = mid; else hi = mid - 1;
+            }
+            b = lo;
+            i = row - a.batches[b].q_off;
+        }
+        const BatchInfo bi = a.batches[b];
+        if (i >= 0 && i < bi.Sq) {
+            int nv = bi.Sk;
+            if (a.mode == 3) {
+                int lim = i + 1 + bi.Sk - bi.Sq;
+                nv = lim < 0 ? 0 : (lim < bi.Sk ? lim : bi.Sk);
+            }
+            n = nv;
+        }
+    }
+    int32_t *oidx = a.out_idx + (int64_t)row * k;
+    float *oval = a.out_val ? a.out_val + (int64_t)row * k : nullptr;
+    const int m = n < k ? n : k;
+
+    if (m == 0) {
+        for (int j = tid; j < k; j += kTopkThreads) {
+            oidx[j] = -1;
+            if (oval) oval[j] = __uint_as_float(0xFF800000u);
+        }
+        return;
+    }
+
+    uint32_t *hist = reinterpret_cast<uint32_t *>(smem);              // 4096 words
+    uint32_t *keyA = hist + 4096;
+    int32_t *idxA = reinterpret_cast<int32_t *>(keyA + a.kmax);
+    uint32_t *keyB = reinterpret_cast<uint32_t *>(idxA + a.kmax);
+    int32_t *idxB = reinterpret_cast<int32_t *>(keyB + a.kmax);
+    uint32_t *cache = reinterpret_cast<uint32_t *>(idxB + a.kmax);
+
+    RowSrc src;
+    src.g = a.scores + (int64_t)row * a.ld;
+    src.c = nullptr;
+    src.n = n;
+    const int n4 = (n + 3) >> 2;
+    if (n <= a.cap) {
+        const float4 *g4 = reinterpret_cast<const float4 *>(src.g);
+        uint4 *c4 = reinterpret_cast<uint4 *>(cache);
+        for (int j4 = tid; j4 < n4; j4 += kTopkThreads) {
+            float4 v = g4[j4];
+            c4[j4] = make_uint4(to_key(v.x), to_key(v.y), to_key(v.z), to_key(v.w));
+        }
+        src.c = cache;
+        __syncthreads();
+    }
+
+    // --- 1. radix select of the k-th largest key (only when n > k)
+    uint32_t T = 0;
+    int need_eq = 0;
+    if (n > k) {
+        uint32_t prefix = 0, pmask = 0;
+        int remaining = k;
+        const int shifts[3] = {21, 10, 0};
+        const int widths[3] = {11, 11, 10};
+#pragma unroll
+        for (int pass = 0; pass < 3; ++pass) {
+            const int shift = shifts[pass], bins = 1 << widths[pass];
+            const uint32_t dmask = (uint32_t)bins - 1u;
+            for (int j = tid; j < bins; j += kTopkThreads) hist[j] = 0;
+            __syncthreads();
+            // every lane runs the same number of iterations (match_any below)
+            for (int base4 = 0; base4 < n4; base4 += kTopkThreads) {
+                const int j4 = base4 + tid;
+                uint32_t kv[4] = {0, 0, 0, 0};
+                if (j4 < n4) {
+                    uint4 q = src.load4(j4);
+                    kv[0] = q.x; kv[1] = q.y; kv[2] = q.z; kv[3] = q.w;
+                }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = j4 * 4 + e;
+                    const bool act = j < n && (kv[e] & pmask) == prefix;
+                    const uint32_t d = act ? (kv[e] >> shift) & dmask : 0xFFFFFFFFu;
+                    const uint32_t peers = __match_any_sync(0xffffffffu, d);
+                    if (act && (peers & lanemask_lt()) == 0)
+                        atomicAdd(&hist[d], (uint32_t)__popc(peers));
+                }
+            }
+            __syncthreads();
+            // thread t owns `per` consecutive bins, counted from the top digit down
+            const int per = bins / kTopkThreads;
+            uint32_t c = 0;
+            for (int e = 0; e < per; ++e) c += hist[bins - 1 - (tid * per + e)];
+            uint32_t tot;
+            uint32_t above = block_exclusive_scan<uint32_t>(c, s_tmp32, tot);
+            if (above < (uint32_t)remaining && above + c >= (uint32_t)remaining) {
+                uint32_t acc = above;
+                for (int e = 0; e < per; ++e) {
+                    const int d = bins - 1 - (tid * per + e);
+                    const uint32_t h = hist[d];
+                    if (acc + h >= (uint32_t)remaining) {
+                        s_digit = (uint32_t)d;
+                        s_above = acc;
+                        break;
+                    }
+                    acc += h;
+                }
+            }
+            __syncthreads();
+            remaining -= (int)s_above;
+            prefix |= s_digit << shift;
+            pmask |= dmask << shift;
+            __syncthreads();
+        }
+        T = prefix;
+        need_eq = remaining;
+    }
+
+    // --- 2. compaction in index order into keyA/idxA
+    if (n <= k) {
+        for (int j4 = tid; j4 < n4; j4 += kTopkThreads) {
+            uint4 q = src.load4(j4);
+            uint32_t kv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int j = j4 * 4 + e;
+                if (j < n) { keyA[j] = kv[e]; idxA[j] = j; }
+            }
+        }
+    } else {
+        uint32_t gt_carry = 0, eq_carry = 0;
+        for (int base4 = 0; base4 < n4; base4 += kTopkThreads) {
+            const int j4 = base4 + tid;
+            uint32_t kv[4] = {0, 0, 0, 0};
+            uint32_t ngt = 0, neq = 0;
+            if (j4 < n4) {
+                uint4 q = src.load4(j4);
+                kv[0] = q.x; kv[1] = q.y; kv[2] = q.z; kv[3] = q.w;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = j4 * 4 + e;
+                    if (j < n) { ngt += kv[e] > T; neq += kv[e] == T; }
+                }
+            }
+            uint64_t packed = ((uint64_t)neq << 32) | ngt, tot;
+            uint64_t before = block_exclusive_scan<uint64_t>(packed, s_tmp64, tot);
+            uint32_t gt_b = gt_carry + (uint32_t)before;
+            uint32_t eq_b = eq_carry + (uint32_t)(before >> 32);
+            if (j4 < n4) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = j4 * 4 + e;
+                    if (j >= n) break;
+                    const bool gt = kv[e] > T, eq = kv[e] == T;
+                    if (gt || (eq && eq_b < (uint32_t)need_eq)) {
+                        const uint32_t pos = gt_b + (eq_b < (uint32_t)need_eq ? eq_b : (uint32_t)need_eq);
+                        keyA[pos] = kv[e];
+                        idxA[pos] = j;
+                    }
+                    gt_b += gt;
+                    eq_b += eq;
+                }
+            }
+            gt_carry += (uint32_t)tot;
+            eq_carry += (uint32_t)(tot >> 32);
+        }
+    }
+    __syncthreads();
+
+    // --- 3. stable LSB radix sort of keyA/idxA (m elements) by descending key
+    uint32_t *kin = keyA, *kout = keyB;
+    int32_t *iin = idxA, *iout = idxB;
+    if (m > 1) {
+        if (tid == 0) { s_or = 0; s_and = 0xFFFFFFFFu; }
+        __syncthreads();
+        uint32_t vor = 0, vand = 0xFFFFFFFFu;
+        for (int j = tid; j < m; j += kTopkThreads) { vor |= kin[j]; vand &= kin[j]; }
+        atomicOr(&s_or, vor);
+        atomicAnd(&s_and, vand);
+        __syncthreads();
+        const uint32_t diff = s_or ^ s_and;
+        const int seg = (((m + kWarps - 1) / kWarps) + 31) & ~31;     // elements per warp
+        const int rounds = seg >> 5;
+        uint32_t *whist = hist + warp * 256;                            // per-warp digit counts
+        for (int shift = 0; shift < 32; shift += 8) {
+            if (((diff >> shift) & 0xFFu) == 0) continue;               // same digit everywhere
+            for (int j = lane; j < 256; j += 32) whist[j] = 0;
+            __syncwarp();
+            uint32_t local[kSortMaxRounds];
+            const int wbeg = warp * seg;
+#pragma unroll
+            for (int r = 0; r < kSortMaxRounds; ++r) {
+                if (r >= rounds) break;
+                const int e = wbeg + r * 32 + lane;
+                const bool valid = e < m;
+                const uint32_t d = valid ? ((~kin[e]) >> shift) & 0xFFu : 0xFFFFFFFFu;
+                const uint32_t peers = __match_any_sync(0xffffffffu, d);
+                uint32_t cnt = 0;
+                if (valid) cnt = whist[d];
+                local[r] = cnt + __popc(peers & lanemask_lt());
+                __syncwarp();
+                if (valid && (peers & lanemask_lt()) == 0) whist[d] = cnt + __popc(peers);
+                __syncwarp();
+            }
+            __syncthreads();
+            // exclusive scan over (digit major, warp minor): thread t owns digit t>>1,
+            // warps (t&1)*8 .. +8
+            const int d0 = tid >> 1, w0 = (tid & 1) * 8;
+            uint32_t own[8], sum = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) { own[j] = hist[(w0 + j) * 256 + d0]; sum += own[j]; }
+            uint32_t tot;
+            uint32_t off = block_exclusive_scan<uint32_t>(sum, s_tmp32, tot);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) { hist[(w0 + j) * 256 + d0] = off; off += own[j]; }
+            __syncthreads();
+#pragma unroll
+            for (int r = 0; r < kSortMaxRounds; ++r) {
+                if (r >= rounds) break;
+                const int e = wbeg + r * 32 + lane;
+                if (e < m) {
+                    const uint32_t kk = kin[e];
+                    const uint32_t d = ((~kk) >> shift) & 0xFFu;
+                    const uint32_t dst = whist[d] + local[r];
+                    kout[dst] = kk;
+                    iout[dst] = iin[e];
+                }
+            }
+            __syncthreads();
+            uint32_t *tk = kin; kin = kout; kout = tk;
+            int32_t *ti = iin; iin = iout; iout = ti;
+        }
+    }
+
+    // --- 4. write out
+    for (int j = tid; j < k; j += kTopkThreads) {
+        if (j < m) {
+            oidx[j] = iin[j];
+            if (oval) oval[j] = from_key(kin[j]);
+        } else {
+            oidx[j] = -1;
+            if (oval) oval[j] = __uint_as_float(0xFF800000u);
+        }
+    }
+}
+
+}  // namespace
+
+size_t topk_smem_bytes(int cap, int kmax)
+{
+    return (size_t)4096 * 4 + (size_t)kmax * 16 + (size_t)((cap + 3) & ~3) * 4;
+}
+
+cudaError_t launch_topk(const TopkArgs &a, cudaStream_t s)
+{
+    const size_t smem = topk_smem_bytes(a.cap, a.kmax);
+    cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    if (a.rows <= 0) return cudaSuccess;
+    topk_kernel<<<a.rows, kTopkThreads, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace li

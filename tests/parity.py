@@ -1,0 +1,92 @@
+"""Element-by-element comparison of the CUDA path with the fp64 oracle.
+
+The rule (tolerance |g - o| <= atol + rtol*|o|; bf16/fp16: rtol 2e-3, atol
+1e-4; fp8: rtol 5e-2, atol 1e-4):
+  * slots past min(k, visible) hold index -1 and value -inf, bit for bit;
+  * the valid indices are distinct and visible (0 <= t < nvis);
+  * values are non-increasing, each within tolerance of the oracle's score of
+    that key and of the oracle's value in the same slot;
+  * every key whose oracle score exceeds s_k + tol(s_k) is selected, and every
+    selected key has an oracle score >= s_k - tol(s_k), where s_k is the
+    oracle's k-th value: swaps are allowed only inside the tolerance band
+    around the k-th score.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+
+TOL = {"bf16": (2e-3, 1e-4), "fp16": (2e-3, 1e-4), "e4m3": (5e-2, 1e-4)}
+NEG_INF_BITS = np.float32(-np.inf).view(np.uint32)
+
+
+def to_device(inputs, device="cuda"):
+    return {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in inputs.items()}
+
+
+def compare_rows(p, gpu_idx, gpu_val, orc, rows_label=None, rtol=None, atol=None):
+    """gpu_idx/gpu_val: numpy [n, k] for the rows the oracle evaluated (orc)."""
+    if rtol is None:
+        rtol, atol = TOL[p.dtype_qk]
+    k = p.sparse_count
+    scores = orc["scores"]
+    for r in range(gpu_idx.shape[0]):
+        label = rows_label[r] if rows_label is not None else r
+        nv = int(orc["nvis"][r])
+        m = min(k, nv)
+        gi = gpu_idx[r]
+        assert np.all(gi[m:] == -1), "row %s: padding indices" % label
+        if gpu_val is not None:
+            gv = gpu_val[r]
+            assert np.all(gv[m:].view(np.uint32) == NEG_INF_BITS), "row %s: padding values" % label
+        if m == 0:
+            continue
+        sel = gi[:m].astype(np.int64)
+        assert np.all(sel >= 0) and np.all(sel < nv), "row %s: index out of the visible range" % label
+        assert len(np.unique(sel)) == m, "row %s: duplicate indices" % label
+        s = scores[r]
+        os_sorted = orc["v64"][r][:m]
+        s_k = os_sorted[m - 1]
+        tol_k = atol + rtol * abs(s_k)
+        got_s = s[sel]
+        assert np.all(np.isfinite(got_s)), "row %s: selected an invisible key" % label
+        assert np.all(got_s >= s_k - tol_k), (
+            "row %s: selected key below the k-th score band (min %.6g < %.6g)"
+            % (label, got_s.min(), s_k - tol_k))
+        must = np.nonzero(s[:nv] > s_k + tol_k)[0]
+        missing = np.setdiff1d(must, sel)
+        assert missing.size == 0, "row %s: missed keys %s" % (label, missing[:8])
+        if gpu_val is not None:
+            gv = gpu_val[r][:m].astype(np.float64)
+            assert np.all(np.diff(gv) <= 0), "row %s: values not non-increasing" % label
+            err_key = np.abs(gv - got_s) - (atol + rtol * np.abs(got_s))
+            assert np.all(err_key <= 0), "row %s: value vs key score off by %.3g (slot %d)" % (
+                label, np.abs(gv - got_s)[np.argmax(err_key)], int(np.argmax(err_key)))
+            err_slot = np.abs(gv - os_sorted) - (atol + rtol * np.abs(os_sorted))
+            assert np.all(err_slot <= 0), "row %s: value vs sorted oracle off by %.3g (slot %d)" % (
+                label, np.abs(gv - os_sorted)[np.argmax(err_slot)], int(np.argmax(err_slot)))
+
+
+def check_against_oracle(p, inputs, gpu_idx, gpu_val, rows=None, nthreads=0):
+    """Run the oracle on `rows` (all when None) and compare. gpu_* are full [R, k]."""
+    gi = gpu_idx.reshape(p.rows, p.sparse_count)
+    gv = gpu_val.reshape(p.rows, p.sparse_count) if gpu_val is not None else None
+    orc = oracle.run(p, inputs, rows=rows, want_scores=True, nthreads=nthreads)
+    if rows is not None:
+        gi = gi[np.asarray(rows)]
+        gv = gv[np.asarray(rows)] if gv is not None else None
+    compare_rows(p, gi, gv, orc, rows_label=rows)
+    return orc
+
+
+def sample_rows(p, n_random=256, seed=0, edge=64):
+    """First/last rows, rows around index k and a seeded random sample."""
+    R = p.rows
+    k = p.sparse_count
+    rs = set(range(min(edge, R))) | set(range(max(0, R - edge), R))
+    rs |= set(range(max(0, k - 8), min(R, k + 8)))
+    g = np.random.default_rng(seed)
+    rs |= set(g.integers(0, R, size=min(n_random, R)).tolist())
+    return sorted(rs)

@@ -1,0 +1,234 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Small cases span several 128-key tiles with ragged tails and cover every
+layout pair, both sparse modes, bf16/fp16/fp8, head counts that need padding,
+paged block sizes 16..1024 (also non-contiguous pools), padding rows and rows
+with no visible key.  Exact-integer cases must match the oracle bit for bit
+(indices, including lower-index tie-breaks, and values).  The named workloads
+run at full size: completely where the oracle is fast enough, else on a
+seeded row sample.
+"""
+from __future__ import annotations
+
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_attention_top_n1_b200 as li
+import synth
+from parity import check_against_oracle, sample_rows, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def run_gpu(p, inputs):
+    d = to_device(inputs)
+    pr = li.make_params(p)
+    ws = li.alloc_workspace(pr)
+    idx, val = li.indexer(pr, d["query"], d["key"], d["weights"], act_seq_q=d.get("act_q"),
+                          act_seq_k=d.get("act_k"), block_table=d.get("block_table"),
+                          q_scale=d.get("q_scale"), k_scale=d.get("k_scale"), workspace=ws)
+    assert li.li_last_launch_count() == 3
+    flags = li.li_read_device_status(ws)
+    torch.cuda.synchronize()
+    gi = idx.cpu().numpy().reshape(p.rows, p.sparse_count)
+    gv = val.cpu().numpy().reshape(p.rows, p.sparse_count) if p.return_value else None
+    return gi, gv, flags
+
+
+def small(seed, **kw):
+    base = dict(B=2, S1=40, S2=300, N1=8, D=128, sparse_count=64, return_value=1)
+    base.update(kw)
+    return synth.make_random(seed, **base)
+
+
+CASES = {
+    "bsnd_mode0": dict(sparse_mode=0),
+    "bsnd_mode3": dict(sparse_mode=3),
+    "bsnd_mode3_full": dict(sparse_mode=3, ragged=False, S1=300),
+    "bsnd_fp16_d64_n32": dict(dtype_qk="fp16", dtype_w="fp32", D=64, N1=32, sparse_mode=0),
+    "bsnd_n64": dict(N1=64, S1=20, sparse_mode=3),
+    "bsnd_n3_padded_heads": dict(N1=3, sparse_mode=3),
+    "bsnd_n17_padded_heads": dict(N1=17, sparse_mode=0, dtype_w="fp16"),
+    "bsnd_n1": dict(N1=1, sparse_mode=3, S1=70),
+    "bsnd_k1": dict(sparse_count=1, sparse_mode=3),
+    "bsnd_k_over_visible": dict(sparse_count=400, sparse_mode=3),
+    "bsnd_empty_rows": dict(empty_rows=True, B=4, sparse_mode=3),
+    "bsnd_q_longer_than_k": dict(S1=300, S2=100, ragged=False, sparse_mode=3),
+    "tnd_mode3": dict(layout_q="TND", layout_k="TND", sparse_mode=3, B=3),
+    "tnd_mode0": dict(layout_q="TND", layout_k="TND", sparse_mode=0, B=3),
+    "pa16": dict(layout_k="PA_BSND", block_size=16, sparse_mode=3),
+    "pa48": dict(layout_k="PA_BSND", block_size=48, sparse_mode=3),
+    "pa64_strided": dict(layout_k="PA_BSND", block_size=64, key_block_pad=8, sparse_mode=3),
+    "pa128": dict(layout_k="PA_BSND", block_size=128, sparse_mode=0, S2=700),
+    "pa256": dict(layout_k="PA_BSND", block_size=256, sparse_mode=3, S2=700),
+    "pa1024": dict(layout_k="PA_BSND", block_size=1024, sparse_mode=3, S2=1500),
+    "tnd_q_pa_k": dict(layout_q="TND", layout_k="PA_BSND", block_size=32, sparse_mode=0),
+    "decode_pa": dict(layout_k="PA_BSND", block_size=128, S1=1, ragged=False, sparse_mode=3,
+                      N1=64, S2=1000, B=5),
+    "quant_tnd": dict(layout_q="TND", layout_k="TND", quant=True, dtype_w="fp32", N1=64,
+                      S1=60, S2=300, sparse_mode=3),
+    "quant_pa": dict(layout_k="PA_BSND", quant=True, dtype_w="fp32", block_size=64, N1=64,
+                     sparse_mode=3),
+    "quant_bsnd_n8": dict(quant=True, dtype_w="fp32", sparse_mode=0),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_small_case_parity(name):
+    p, inp = small(zlib.crc32(name.encode()) % 1000, **CASES[name])
+    gi, gv, flags = run_gpu(p, inp)
+    assert flags == 0
+    check_against_oracle(p, inp, gi, gv)
+
+
+@pytest.mark.parametrize("name", ["bsnd_mode3", "bsnd_fp16_d64_n32", "tnd_mode3", "pa48",
+                                  "bsnd_n3_padded_heads", "quant_tnd", "quant_pa", "decode_pa"])
+def test_exact_integer_parity(name):
+    """Small-integer inputs: every product and sum is exact in fp32, so the GPU
+    must reproduce the oracle exactly, ties broken toward the lower index."""
+    p, inp = small(500 + len(name), **CASES[name])
+    g = torch.Generator().manual_seed(7)
+    inp = dict(inp)
+    for key in ("query", "key", "weights"):
+        t = inp[key]
+        inp[key] = torch.randint(-3, 4, t.shape, generator=g).to(torch.float32).to(t.dtype)
+    if p.quant:
+        for key in ("q_scale", "k_scale"):
+            e = torch.randint(-2, 3, inp[key].shape, generator=g).to(torch.float32)
+            inp[key] = torch.pow(2.0, e)
+    gi, gv, flags = run_gpu(p, inp)
+    assert flags == 0
+    o = oracle.run(p, inp)
+    np.testing.assert_array_equal(gi, o["idx"])
+    np.testing.assert_array_equal(gv, o["val"])
+
+
+def test_tiny_workload():
+    p, inp = synth.make_tiny()
+    gi, gv, flags = run_gpu(p, inp)
+    assert flags == 0
+    check_against_oracle(p, inp, gi, gv)
+
+
+def test_cfg2_workload_full():
+    p, inp = synth.make_cfg2()
+    gi, gv, flags = run_gpu(p, inp)
+    assert flags == 0
+    check_against_oracle(p, inp, gi, gv)
+
+
+def test_dsa_prefill_workload_sampled():
+    p, inp = synth.make_dsa_prefill()
+    gi, gv, flags = run_gpu(p, inp)
+    assert flags == 0
+    check_against_oracle(p, inp, gi, gv, rows=sample_rows(p, n_random=96, edge=24))
+
+
+def test_paged_decode_workload_full():
+    p, inp = synth.make_paged_decode(return_value=1)
+    gi, gv, flags = run_gpu(p, inp)
+    assert flags == 0
+    check_against_oracle(p, inp, gi, gv)
+
+
+def test_quant_varlen_workload_sampled():
+    p, inp = synth.make_quant_varlen(return_value=1)
+    gi, gv, flags = run_gpu(p, inp)
+    assert flags == 0
+    cq = [0] + inp["act_q"].tolist()
+    rows = set(sample_rows(p, n_random=64, edge=16))
+    for b in range(p.B):                      # both ends of every sequence
+        rows |= {cq[b], cq[b] + 1, cq[b + 1] - 2, cq[b + 1] - 1}
+    check_against_oracle(p, inp, gi, gv, rows=sorted(rows))
+
+
+# ------------------------------------------------------------------ Top-k stage alone
+
+def _topk_reference(rows_np, lens, k):
+    R = rows_np.shape[0]
+    idx = np.full((R, k), -1, dtype=np.int32)
+    val = np.full((R, k), -np.inf, dtype=np.float32)
+    for r in range(R):
+        n = lens[r]
+        v = rows_np[r, :n]
+        order = np.lexsort((np.arange(n), -v.astype(np.float64)))[:k]
+        idx[r, :len(order)] = order
+        val[r, :len(order)] = v[order]
+    return idx, val
+
+
+@pytest.mark.parametrize("ld,k,quantised", [(4096, 1024, False), (300, 64, True),
+                                            (8192, 2048, True), (40000, 2048, False),
+                                            (40000, 512, True), (64, 100, False)])
+def test_topk_stage_exact(ld, k, quantised):
+    g = torch.Generator().manual_seed(ld + k)
+    R = 12
+    x = torch.randn(R, ld, generator=g)
+    if quantised:                                   # many exact ties, +0 and -0
+        x = torch.round(x * 4) / 4
+        x[:, ::7] = -0.0
+    lens = torch.randint(1, ld + 1, (R,), generator=g).to(torch.int32)
+    lens[0] = ld
+    lens[1] = min(k, ld)
+    d = x.cuda()
+    idx = torch.empty(R, k, dtype=torch.int32, device="cuda")
+    val = torch.empty(R, k, dtype=torch.float32, device="cuda")
+    li.li_topk(d, ld, lens.cuda(), R, k, idx, val)
+    torch.cuda.synchronize()
+    ri, rv = _topk_reference(x.numpy(), lens.numpy(), k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ri)
+    np.testing.assert_array_equal(val.cpu().numpy(), rv)
+
+
+# ------------------------------------------------------------------ device status word
+
+def test_device_flags_bad_lengths_and_blocks():
+    p, inp = small(3, layout_k="PA_BSND", block_size=64, sparse_mode=3)
+    inp = dict(inp)
+    bt = inp["block_table"].clone()
+    bt[0, 0] = p.num_blocks + 5                      # outside the pool: skipped, flagged
+    inp["block_table"] = bt
+    _, _, flags = run_gpu(p, inp)
+    assert flags & li.DEV_BAD_BLOCK
+    p2, inp2 = small(4, sparse_mode=3)
+    inp2 = dict(inp2)
+    ak = inp2["act_k"].clone()
+    ak[1] = p2.S2 + 10                               # longer than the key tensor: clamped
+    inp2["act_k"] = ak
+    _, _, flags = run_gpu(p2, inp2)
+    assert flags & li.DEV_BAD_KLEN
+
+
+def test_device_flags_negative_scale():
+    p, inp = small(5, layout_q="TND", layout_k="TND", quant=True, dtype_w="fp32",
+                   sparse_mode=3)
+    inp = dict(inp)
+    ks = inp["k_scale"].clone()
+    ks[3] = -1.0
+    inp["k_scale"] = ks
+    _, _, flags = run_gpu(p, inp)
+    assert flags & li.DEV_NEG_SCALE
+
+
+def test_bounded_wait_expires_and_context_survives():
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    li.li_selftest_bounded_wait(status, 5_000_000)    # 5 ms, nothing ever arrives
+    torch.cuda.synchronize()
+    assert int(status.item()) & li.DEV_TIMEOUT
+    # the context is still usable afterwards
+    p, inp = synth.make_tiny()
+    gi, gv, flags = run_gpu(p, inp)
+    assert flags == 0
+    check_against_oracle(p, inp, gi, gv)
+
+
+def test_repeat_calls_are_deterministic():
+    p, inp = small(9, sparse_mode=3, N1=64, S1=64, S2=700)
+    a = run_gpu(p, inp)
+    b = run_gpu(p, inp)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])

@@ -333,6 +333,9 @@ def main():
     starts = [mk() for _ in range(K)]
     ends = [mk() for _ in range(K)]
     prof = [[mk() for _ in range(4)] for _ in range(K)]
+    for e in [x for row in prof for x in row]:      # torch creates events lazily
+        e.record()
+    torch.cuda.synchronize()
     clocks = ClockSampler(local)
     clocks.start()
     barrier()

@@ -26,9 +26,9 @@ thread_local int32_t g_launches = 0;
 thread_local cudaEvent_t g_prof[4] = {nullptr, nullptr, nullptr, nullptr};
 thread_local bool g_prof_on = false;
 
-void prof_mark(int i, cudaStream_t s)
+bool prof_mark(int i, cudaStream_t s)
 {
-    if (g_prof_on) cudaEventRecord(g_prof[i], s);
+    return !g_prof_on || cudaEventRecord(g_prof[i], s) == cudaSuccess;
 }
 
 li_status fail(li_status s, const char *fmt, ...)
@@ -307,11 +307,11 @@ li_status run(const li_params *pp, bool quant, const void *query, const void *ke
     pa.max_blocks = w.max_blocks;
     pa.ld = w.ld;
     pa.pa_capacity = (int64_t)p.max_blocks_per_seq * p.block_size;
-    prof_mark(0, s);
+    if (!prof_mark(0, s)) return fail(LI_ERR_CUDA, "recording profile event 0 failed");
     cudaError_t e = launch_plan(pa, s);
     if (e != cudaSuccess) return fail(LI_ERR_CUDA, "scheduler launch: %s", cudaGetErrorString(e));
     ++g_launches;
-    prof_mark(1, s);
+    if (!prof_mark(1, s)) return fail(LI_ERR_CUDA, "recording profile event 1 failed");
 
     ScoreArgs sa{};
     sa.weights = weights;
@@ -339,7 +339,7 @@ li_status run(const li_params *pp, bool quant, const void *query, const void *ke
     e = launch_score(sa, t, qmap, kmap, quant ? 1 : 0, sms, s);
     if (e != cudaSuccess) return fail(LI_ERR_CUDA, "score launch: %s", cudaGetErrorString(e));
     ++g_launches;
-    prof_mark(2, s);
+    if (!prof_mark(2, s)) return fail(LI_ERR_CUDA, "recording profile event 2 failed");
 
     TopkArgs ta{};
     ta.scores = scores;
@@ -360,7 +360,7 @@ li_status run(const li_params *pp, bool quant, const void *query, const void *ke
     e = launch_topk(ta, s);
     if (e != cudaSuccess) return fail(LI_ERR_CUDA, "top-k launch: %s", cudaGetErrorString(e));
     ++g_launches;
-    prof_mark(3, s);
+    if (!prof_mark(3, s)) return fail(LI_ERR_CUDA, "recording profile event 3 failed");
     return LI_OK;
 }
 

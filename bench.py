@@ -320,9 +320,18 @@ def main():
 
     args_dev = (d["query"], d["key"], d["weights"], d.get("q_scale"), d.get("k_scale"),
                 d.get("act_q"), d.get("act_k"), d.get("block_table"), idx, val)
-    for _ in range(args.warmup):
+    clocks = ClockSampler(local)
+    clocks.start()
+    # W warm-up steps, then more of the same until the clock sampler has seen
+    # the GPU under this load for a while (its period is 200 ms)
+    t_warm = time.perf_counter()
+    nwarm = 0
+    while nwarm < args.warmup or time.perf_counter() - t_warm < 0.8:
         flush.zero_()
         call(*args_dev)
+        nwarm += 1
+        if nwarm % 16 == 0:
+            torch.cuda.synchronize()
     torch.cuda.synchronize()
     flags = li.li_read_device_status(wsb)
     if flags:
@@ -336,8 +345,6 @@ def main():
     for e in [x for row in prof for x in row]:      # torch creates events lazily
         e.record()
     torch.cuda.synchronize()
-    clocks = ClockSampler(local)
-    clocks.start()
     barrier()
     torch.cuda.synchronize()
     launches = 0

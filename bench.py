@@ -281,6 +281,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--plain", action="store_true",
+                    help="exactly W warm-up and K timed calls, no clock sampling, e2e or "
+                         "CPU baseline (a fixed launch sequence for ncu)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -321,12 +324,13 @@ def main():
     args_dev = (d["query"], d["key"], d["weights"], d.get("q_scale"), d.get("k_scale"),
                 d.get("act_q"), d.get("act_k"), d.get("block_table"), idx, val)
     clocks = ClockSampler(local)
-    clocks.start()
+    if not args.plain:
+        clocks.start()
     # W warm-up steps, then more of the same until the clock sampler has seen
     # the GPU under this load for a while (its period is 200 ms)
     t_warm = time.perf_counter()
     nwarm = 0
-    while nwarm < args.warmup or time.perf_counter() - t_warm < 0.8:
+    while nwarm < args.warmup or (not args.plain and time.perf_counter() - t_warm < 0.8):
         flush.zero_()
         call(*args_dev)
         nwarm += 1
@@ -398,7 +402,7 @@ def main():
     # end to end through the C ABI with host buffers: H2D of the inputs from
     # pinned memory, the call, D2H of the outputs, all inside the timed region
     e2e = None
-    if not args.no_e2e:
+    if not (args.no_e2e or args.plain):
         host = {k: v.pin_memory() for k, v in inp.items()}
         hidx = torch.empty(shape, dtype=torch.int32).pin_memory()
         hval = torch.empty(shape, dtype=torch.float32).pin_memory() if p.return_value else None
@@ -425,7 +429,7 @@ def main():
         raise SystemExit("device status 0x%x after timing" % flags)
 
     cpu = None
-    if rank == 0 and n == 1 and not args.no_cpu_baseline:
+    if rank == 0 and n == 1 and not (args.no_cpu_baseline or args.plain):
         cpu, _, _ = cpu_oracle_sample(p, inp)
 
     dtype = {"bf16": "bf16", "fp16": "fp16", "e4m3": "fp8_e4m3"}[p.dtype_qk]

@@ -9,8 +9,9 @@
 //
 // Output (in the workspace):
 //   BatchInfo[b]  clamped lengths and offsets of every batch
-//   BlockInfo[g]  query block g: its batch, first query, first unit and the
-//                 number of key tiles its last (most-seeing) query needs
+//   BlockInfo[g]  query block g: its batch, first query, the number of key
+//                 tiles its last (most-seeing) query needs, and its first
+//                 position in the weighted work list (tiles + kQCost per block)
 //   PlanHeader    totals and the device status word (cleared here: this is
 //                 the first kernel of every call)
 // Lengths outside what the tensors or the declared bounds can hold are
@@ -156,10 +157,12 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a)
             blk.i0 = i0;
             blk.ntiles = ntiles;
         }
-        int32_t incl = ntiles;
+        // a block weighs its key tiles plus the cost of loading its query tile
+        const int32_t weight = ntiles > 0 ? ntiles + kQCost : 0;
+        int32_t incl = weight;
         const int32_t tot = block_inclusive_scan(incl, s_tmp);
         if (g < total_blocks) {
-            blk.unit_start = carry + incl - ntiles;
+            blk.unit_start = carry + incl - weight;
             a.blocks[g] = blk;
         }
         carry += tot;

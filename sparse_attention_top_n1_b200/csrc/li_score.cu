@@ -51,33 +51,71 @@ struct Geometry {
                                    NBARS * 8 + 16;
 };
 
-// Walks the flat unit list: unit u -> (query block qb, key tile).
+// Walks this CTA's share [w0, w1) of the weighted work list.  A block of n
+// key tiles occupies n + kQCost consecutive positions: kQCost for loading its
+// query tile, then one per key tile; a tile belongs to the CTA whose range
+// holds its position, so every tile is processed exactly once.
 struct Walker {
     const BlockInfo *blocks;
-    int nblocks;
-    int qb, tile, ntiles;
-    __device__ void init(int u)
+    int nblocks, w_end;
+    int qb, tile, ntiles, start;
+    __device__ void load_block()
     {
-        int lo = 0, hi = nblocks - 1;                  // last block with unit_start <= u
+        if (qb < nblocks) {
+            start = blocks[qb].unit_start;
+            ntiles = blocks[qb].ntiles;
+        }
+    }
+    __device__ void normalize()
+    {
+        while (qb < nblocks && tile >= ntiles) {
+            ++qb;
+            tile = 0;
+            load_block();
+        }
+    }
+    __device__ void init(int w0, int w1)
+    {
+        w_end = w1;
+        int lo = 0, hi = nblocks - 1;                  // last block starting at or before w0
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
-            if (blocks[mid].unit_start <= u) lo = mid; else hi = mid - 1;
+            if (blocks[mid].unit_start <= w0) lo = mid; else hi = mid - 1;
         }
         qb = lo;
-        tile = u - blocks[lo].unit_start;
-        ntiles = blocks[lo].ntiles;
+        load_block();
+        tile = w0 - start - kQCost;
+        if (tile < 0) tile = 0;
+        normalize();
     }
+    __device__ bool valid() const { return qb < nblocks && start + kQCost + tile < w_end; }
     __device__ void next()
     {
-        if (++tile >= ntiles) {
-            tile = 0;
-            do {
-                ++qb;
-                ntiles = qb < nblocks ? blocks[qb].ntiles : 1;
-            } while (ntiles == 0);
-        }
+        ++tile;
+        normalize();
     }
 };
+
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t pack2(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ float hsum2(uint64_t r)
+{
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+    return lo + hi;
+}
 
 __device__ __forceinline__ float load_weight(const void *w, int dtype, int64_t i)
 {
@@ -94,7 +132,7 @@ __device__ __forceinline__ void fail(PlanHeader *hdr, volatile int *abort_flag, 
 }
 
 template <int CHUNKS, int N1P, bool FP8>
-__global__ void __launch_bounds__(kScoreThreads, 1)
+__global__ void __maxnreg__(200)
     score_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                  const ScoreArgs a)
 {
@@ -102,7 +140,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     constexpr int STAGES = G::STAGES;
     constexpr int NQ = 256 / N1P;                 // queries per block
     constexpr int QPW = 128 / N1P;                // queries per epilogue warp half
-    constexpr int NP = N1P >= 32 ? 4 : (N1P == 16 ? 2 : 1);   // partial sums per query
+    constexpr int NP2 = N1P >= 32 ? 4 : (N1P == 16 ? 2 : 1);  // packed partial sums per query
     constexpr int INNER = FP8 ? 128 : 64;         // elements per 128-byte row chunk
 
     extern __shared__ uint8_t smem_raw[];
@@ -157,20 +195,20 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 
     const int total = a.hdr->total_units;
     const int nblocks = a.hdr->total_blocks;
-    const int u_begin = (int)(((int64_t)total * blockIdx.x) / gridDim.x);
-    const int u_end = (int)(((int64_t)total * (blockIdx.x + 1)) / gridDim.x);
+    const int w_begin = (int)(((int64_t)total * blockIdx.x) / gridDim.x);
+    const int w_end = (int)(((int64_t)total * (blockIdx.x + 1)) / gridDim.x);
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0 && u_begin < u_end) {
-            Walker w{a.blocks, nblocks, 0, 0, 0};
-            w.init(u_begin);
+        if (lane == 0 && w_begin < w_end && nblocks > 0) {
+            Walker w{a.blocks, nblocks, 0, 0, 0, 0, 0};
+            w.init(w_begin, w_end);
             int stage = 0, prev_qb = -1;
             uint32_t phase = 0, qphase = 0;
             uint32_t armed = 0, par = 0, q_armed = 0, q_par = 0;
             BlockInfo blk{};
             BatchInfo bi{};
-            for (int u = u_begin; u < u_end; ++u) {
+            for (; w.valid(); w.next()) {
                 if (w.qb != prev_qb) {
                     blk = a.blocks[w.qb];
                     bi = a.batches[blk.b];
@@ -239,7 +277,6 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                     stage = 0;
                     phase ^= 1u;
                 }
-                w.next();
             }
             if (*abort_flag) {
                 // let every copy still in flight land before the CTA exits
@@ -251,14 +288,14 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && u_begin < u_end) {
-            Walker w{a.blocks, nblocks, 0, 0, 0};
-            w.init(u_begin);
+        if (lane == 0 && w_begin < w_end && nblocks > 0) {
+            Walker w{a.blocks, nblocks, 0, 0, 0, 0, 0};
+            w.init(w_begin, w_end);
             int stage = 0, acc = 0, prev_qb = -1;
             uint32_t phase = 0, acc_phase = 0, qphase = 0, idesc = 0;
             bool issued = false;
             const uint32_t sQ_addr = smem_u32(sQ), sK_addr = smem_u32(sK);
-            for (int u = u_begin; u < u_end; ++u) {
+            for (; w.valid(); w.next()) {
                 if (w.qb != prev_qb) {
                     const BlockInfo blk = a.blocks[w.qb];
                     const BatchInfo bi = a.batches[blk.b];
@@ -306,7 +343,6 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                     acc = 0;
                     acc_phase ^= 1u;
                 }
-                w.next();
             }
             if (issued) {
                 // every MMA of this CTA has finished before TMEM is released
@@ -316,19 +352,25 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue
+        // Each thread owns key row `lrow` of the tile and the 128 columns of
+        // its warp half: QPW queries x N1P heads.  Per tile it loads those
+        // columns from TMEM in one go, hands the accumulator back to the MMA
+        // warp, then reduces sum_h W*ReLU(logit) with packed fp32 FMAs.
         const int ew = warp - 2;                   // 0..7
         const int quarter = warp & 3;              // TMEM lanes this warp may access
         const int half = ew >> 2;                  // which 128 of the 256 columns
         const int lrow = quarter * 32 + lane;      // key row within the tile
         float *myW = sW + ew * 128;
-        if (u_begin < u_end) {
-            Walker w{a.blocks, nblocks, 0, 0, 0};
-            w.init(u_begin);
+        if (w_begin < w_end && nblocks > 0) {
+            Walker w{a.blocks, nblocks, 0, 0, 0, 0, 0};
+            w.init(w_begin, w_end);
             int acc = 0, prev_qb = -1, nchunks = 0;
             uint32_t acc_phase = 0;
             BlockInfo blk{};
             BatchInfo bi{};
-            for (int u = u_begin; u < u_end; ++u) {
+            float *row_ptr = nullptr;              // score row of this half's first query
+            int lim0 = 0, nq_valid = 0;            // visible limit of that query; valid queries
+            for (; w.valid(); w.next()) {
                 if (w.qb != prev_qb) {
                     blk = a.blocks[w.qb];
                     bi = a.batches[blk.b];
@@ -336,7 +378,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                     nrows = nrows > NQ ? NQ : nrows;
                     int mine = nrows - half * QPW;     // valid queries of this half
                     mine = mine < 0 ? 0 : (mine > QPW ? QPW : mine);
+                    nq_valid = mine;
                     nchunks = (mine * N1P + 31) / 32;
+                    const int i_first = blk.i0 + half * QPW;
+                    row_ptr = a.scores + (int64_t)(bi.row0 + i_first) * a.ld;
+                    lim0 = a.mode == 3 ? i_first + 1 + bi.Sk - bi.Sq : bi.Sk;
                     __syncwarp();
                     for (int j = lane; j < 128; j += 32) {
                         const int col = half * 128 + j;
@@ -362,6 +408,20 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                     break;
                 }
                 tc_fence_after_sync();
+                const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16) +
+                                      (uint32_t)(acc * kAccCols + half * 128);
+                float v[4][32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    if (c < nchunks) tmem_ld32(trow + c * 32, v[c]);
+                tmem_ld_wait();
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[acc]);
+                if (++acc == kAccStages) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
                 const int t = w.tile * kTileKeys + lrow;
                 float ks = 1.f;
                 if (a.quant && t < bi.Sk) {
@@ -379,59 +439,44 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                         if (ks < 0.f) atomicOr(&a.hdr->status, LI_DEV_NEG_SCALE);
                     }
                 }
-                float part[QPW][NP];
+                uint64_t part[QPW][NP2];
 #pragma unroll
                 for (int q = 0; q < QPW; ++q)
 #pragma unroll
-                    for (int p = 0; p < NP; ++p) part[q][p] = 0.f;
-                const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16) +
-                                      (uint32_t)(acc * kAccCols + half * 128);
+                    for (int p = 0; p < NP2; ++p) part[q][p] = 0ull;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     if (c < nchunks) {
-                        float v[32];
-                        tmem_ld32(trow + c * 32, v);
-                        tmem_ld_wait();
-                        const float4 *w4 = reinterpret_cast<const float4 *>(myW + c * 32);
+                        const uint4 *w4 = reinterpret_cast<const uint4 *>(myW + c * 32);
 #pragma unroll
                         for (int j4 = 0; j4 < 8; ++j4) {
-                            const float4 ww = w4[j4];
-                            const float wj[4] = {ww.x, ww.y, ww.z, ww.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int j = j4 * 4 + e;
-                                const int q = (c * 32 + j) / N1P;
-                                part[q][j % NP] = fmaf(wj[e], fmaxf(v[j], 0.f), part[q][j % NP]);
-                            }
+                            const uint4 ww = w4[j4];
+                            const int j = j4 * 4;
+                            const int q = (c * 32 + j) / N1P;      // same query for j..j+3
+                            const int p0 = (j / 2) % NP2, p1 = (j / 2 + 1) % NP2;
+                            const uint64_t w01 = pack2(__uint_as_float(ww.x), __uint_as_float(ww.y));
+                            const uint64_t w23 = pack2(__uint_as_float(ww.z), __uint_as_float(ww.w));
+                            part[q][p0] = ffma2(w01, pack2(fmaxf(v[c][j], 0.f), fmaxf(v[c][j + 1], 0.f)),
+                                                part[q][p0]);
+                            part[q][p1] = ffma2(w23, pack2(fmaxf(v[c][j + 2], 0.f), fmaxf(v[c][j + 3], 0.f)),
+                                                part[q][p1]);
                         }
                     }
-                }
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&acc_empty[acc]);
-                if (++acc == kAccStages) {
-                    acc = 0;
-                    acc_phase ^= 1u;
                 }
                 // visible keys only: t < nvis(i); the row keeps its visible prefix
 #pragma unroll
                 for (int q = 0; q < QPW; ++q) {
-                    const int i = blk.i0 + half * QPW + q;
-                    if (half * QPW + q < NQ && i < bi.Sq) {
-                        int nv = bi.Sk;
-                        if (a.mode == 3) {
-                            const int lim = i + 1 + bi.Sk - bi.Sq;
-                            nv = lim < 0 ? 0 : (lim < bi.Sk ? lim : bi.Sk);
-                        }
+                    if (q < nq_valid) {
+                        int nv = lim0 + q;
+                        nv = nv < 0 ? 0 : (nv < bi.Sk ? nv : bi.Sk);
                         if (t < nv) {
                             float s = 0.f;
 #pragma unroll
-                            for (int p = 0; p < NP; ++p) s += part[q][p];
-                            a.scores[(int64_t)(bi.row0 + i) * a.ld + t] = s * ks;
+                            for (int p = 0; p < NP2; ++p) s += hsum2(part[q][p]);
+                            row_ptr[(int64_t)q * a.ld + t] = s * ks;
                         }
                     }
                 }
-                w.next();
             }
         }
     }

@@ -94,82 +94,36 @@ struct RowSrc {
     }
 };
 
-__global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a)
+struct TopkSmem {
+    uint32_t *hist;     // 4096 words: radix histograms, or bucket counts + cursors
+    uint32_t *keyA;     // kmax selected keys
+    int32_t *idxA;
+    uint32_t *keyB;     // kmax: radix ping-pong buffer / bucket threshold-bin candidates
+    int32_t *idxB;
+    uint32_t *cache;    // the row as keys, when it fits
+};
+
+struct TopkShared {
+    uint32_t tmp32[kWarps + 1];
+    uint64_t tmp64[kWarps + 1];
+    uint32_t digit, above, vor, vand, kmin, kmax, maxbin;
+};
+
+// ---------------------------------------------------------------- radix path
+// Exact for every input (ties, equal values, any range): three histogram
+// passes find the k-th key, an index-order compaction selects, a stable LSB
+// radix sort orders.  Used when the bucket path declines a row.
+__device__ void radix_topk(const RowSrc &src, int n, int k, int m, const TopkSmem &s,
+                           TopkShared &sh, int32_t *oidx, float *oval)
 {
-    extern __shared__ __align__(16) uint8_t smem[];
-    __shared__ uint32_t s_tmp32[kWarps + 1];
-    __shared__ uint64_t s_tmp64[kWarps + 1];
-    __shared__ uint32_t s_digit, s_above, s_or, s_and;
-
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int row = blockIdx.x;
-    const int k = a.k;
-
-    // --- which elements of which row
-    int n = 0;
-    if (a.standalone) {
-        n = a.row_len ? a.row_len[row] : (int)a.ld;
-        n = n < 0 ? 0 : (n > a.ld ? (int)a.ld : n);
-    } else {
-        int b = -1, i = 0;
-        if (a.layout_q == LI_BSND) {
-            b = row / a.S1;
-            i = row % a.S1;
-        } else {
-            int lo = 0, hi = a.B - 1;               // last batch with q_off <= row
-            while (lo < hi) {
-                int mid = (lo + hi + 1) >> 1;
-                if (a.batches[mid].q_off <= row) lo = mid; else hi = mid - 1;
-            }
-            b = lo;
-            i = row - a.batches[b].q_off;
-        }
-        const BatchInfo bi = a.batches[b];
-        if (i >= 0 && i < bi.Sq) {
-            int nv = bi.Sk;
-            if (a.mode == 3) {
-                int lim = i + 1 + bi.Sk - bi.Sq;
-                nv = lim < 0 ? 0 : (lim < bi.Sk ? lim : bi.Sk);
-            }
-            n = nv;
-        }
-    }
-    int32_t *oidx = a.out_idx + (int64_t)row * k;
-    float *oval = a.out_val ? a.out_val + (int64_t)row * k : nullptr;
-    const int m = n < k ? n : k;
-
-    if (m == 0) {
-        for (int j = tid; j < k; j += kTopkThreads) {
-            oidx[j] = -1;
-            if (oval) oval[j] = __uint_as_float(0xFF800000u);
-        }
-        return;
-    }
-
-    uint32_t *hist = reinterpret_cast<uint32_t *>(smem);              // 4096 words
-    uint32_t *keyA = hist + 4096;
-    int32_t *idxA = reinterpret_cast<int32_t *>(keyA + a.kmax);
-    uint32_t *keyB = reinterpret_cast<uint32_t *>(idxA + a.kmax);
-    int32_t *idxB = reinterpret_cast<int32_t *>(keyB + a.kmax);
-    uint32_t *cache = reinterpret_cast<uint32_t *>(idxB + a.kmax);
-
-    RowSrc src;
-    src.g = a.scores + (int64_t)row * a.ld;
-    src.c = nullptr;
-    src.n = n;
     const int n4 = (n + 3) >> 2;
-    if (n <= a.cap) {
-        const float4 *g4 = reinterpret_cast<const float4 *>(src.g);
-        uint4 *c4 = reinterpret_cast<uint4 *>(cache);
-        for (int j4 = tid; j4 < n4; j4 += kTopkThreads) {
-            float4 v = g4[j4];
-            c4[j4] = make_uint4(to_key(v.x), to_key(v.y), to_key(v.z), to_key(v.w));
-        }
-        src.c = cache;
-        __syncthreads();
-    }
-
-    // --- 1. radix select of the k-th largest key (only when n > k)
+    uint32_t *hist = s.hist, *keyA = s.keyA, *keyB = s.keyB;
+    int32_t *idxA = s.idxA, *idxB = s.idxB;
+    uint32_t *s_tmp32 = sh.tmp32;
+    uint64_t *s_tmp64 = sh.tmp64;
+    uint32_t &s_digit = sh.digit, &s_above = sh.above, &s_or = sh.vor, &s_and = sh.vand;
+    // radix select of the k-th largest key (only when n > k)
     uint32_t T = 0;
     int need_eq = 0;
     if (n > k) {
@@ -347,7 +301,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a)
         }
     }
 
-    // --- 4. write out
+    // write out
     for (int j = tid; j < k; j += kTopkThreads) {
         if (j < m) {
             oidx[j] = iin[j];
@@ -357,6 +311,236 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a)
             if (oval) oval[j] = __uint_as_float(0xFF800000u);
         }
     }
+}
+
+
+// ---------------------------------------------------------------- bucket path
+// Linear value buckets over [min, max] of the row (monotone in the value):
+// one histogram pass finds the bucket holding the m-th largest value, one
+// scatter pass groups the selected elements by bucket, and each element's
+// final rank is its bucket's offset plus its rank inside the bucket, counted
+// by comparing (value desc, index asc) with the bucket's other members.
+// Declines (returns false, uniformly, before writing anything) when a
+// bucket is too full for counting to be cheap or the range is degenerate.
+constexpr int kBuckets = 2048;
+constexpr int kBinLimit = 64;       // largest selected bucket ranked by counting
+constexpr int kCandLimit = 512;     // largest threshold bucket resolved by counting
+
+__device__ __forceinline__ int bucket_of(uint32_t key, float fmin, float scale)
+{
+    const int b = __float2int_rz((from_key(key) - fmin) * scale);
+    return b < 0 ? 0 : (b >= kBuckets ? kBuckets - 1 : b);
+}
+
+__device__ bool bucket_topk(const RowSrc &src, int n, int k, int m, int kmax, const TopkSmem &s,
+                            TopkShared &sh, int32_t *oidx, float *oval)
+{
+    const int tid = threadIdx.x;
+    const float fmin = from_key(sh.kmin), fmax = from_key(sh.kmax);
+    const float range = fmax - fmin;
+    if (!(range > 0.f) || !isfinite(range)) return false;
+    const float scale = (float)kBuckets / range;
+    if (!isfinite(scale)) return false;
+    uint32_t *hist = s.hist, *cur = s.hist + kBuckets;
+    const int n4 = (n + 3) >> 2;
+
+    for (int j = tid; j < kBuckets; j += kTopkThreads) hist[j] = 0;
+    if (tid == 0) sh.maxbin = 0;
+    __syncthreads();
+    for (int j4 = tid; j4 < n4; j4 += kTopkThreads) {
+        const uint4 q = src.load4(j4);
+        const uint32_t kv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            if (j4 * 4 + e < n) atomicAdd(&hist[bucket_of(kv[e], fmin, scale)], 1u);
+    }
+    __syncthreads();
+
+    // buckets from the top down: thread t owns buckets kBuckets-1-(t*per+e)
+    constexpr int per = kBuckets / kTopkThreads;
+    uint32_t c = 0;
+#pragma unroll
+    for (int e = 0; e < per; ++e) c += hist[kBuckets - 1 - (tid * per + e)];
+    uint32_t tot;
+    const uint32_t above_t = block_exclusive_scan<uint32_t>(c, sh.tmp32, tot);
+    uint32_t acc = above_t;
+#pragma unroll
+    for (int e = 0; e < per; ++e) {
+        const int d = kBuckets - 1 - (tid * per + e);
+        const uint32_t h = hist[d];
+        if (acc < (uint32_t)m && acc + h >= (uint32_t)m) {
+            sh.digit = (uint32_t)d;
+            sh.above = acc;
+        }
+        cur[d] = acc;                       // first slot of bucket d
+        acc += h;
+    }
+    __syncthreads();
+    const int bstar = (int)sh.digit;
+    const uint32_t above = sh.above;
+    const uint32_t cstar = hist[bstar];
+    uint32_t lmax = 0;
+#pragma unroll
+    for (int e = 0; e < per; ++e) {
+        const int d = kBuckets - 1 - (tid * per + e);
+        if (d > bstar) lmax = max(lmax, hist[d]);
+    }
+    if (lmax) atomicMax(&sh.maxbin, lmax);
+    __syncthreads();
+    if (sh.maxbin > (uint32_t)kBinLimit || cstar > (uint32_t)min(kCandLimit, kmax)) return false;
+
+    // scatter: selected buckets into keyA/idxA at their bucket slots, the
+    // threshold bucket into keyB/idxB
+    for (int j4 = tid; j4 < n4; j4 += kTopkThreads) {
+        const uint4 q = src.load4(j4);
+        const uint32_t kv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int j = j4 * 4 + e;
+            if (j >= n) break;
+            const int b = bucket_of(kv[e], fmin, scale);
+            if (b > bstar) {
+                const uint32_t pos = atomicAdd(&cur[b], 1u);
+                s.keyA[pos] = kv[e];
+                s.idxA[pos] = j;
+            } else if (b == bstar) {
+                const uint32_t pos = atomicAdd(&cur[b], 1u) - above;
+                s.keyB[pos] = kv[e];
+                s.idxB[pos] = j;
+            }
+        }
+    }
+    __syncthreads();
+
+    // the threshold bucket: keep the `need` best, ranked among themselves
+    const uint32_t need = (uint32_t)m - above;
+    for (uint32_t e = tid; e < cstar; e += kTopkThreads) {
+        const uint32_t kv = s.keyB[e];
+        const int32_t iv = s.idxB[e];
+        uint32_t r = 0;
+        for (uint32_t q = 0; q < cstar; ++q) {
+            const uint32_t kq = s.keyB[q];
+            r += (kq > kv) | ((kq == kv) & (s.idxB[q] < iv));
+        }
+        if (r < need) {
+            oidx[above + r] = iv;
+            if (oval) oval[above + r] = from_key(kv);
+        }
+    }
+    // the buckets above it: bucket offset + rank inside the bucket
+    for (uint32_t p = tid; p < above; p += kTopkThreads) {
+        const uint32_t kv = s.keyA[p];
+        const int32_t iv = s.idxA[p];
+        const int b = bucket_of(kv, fmin, scale);
+        const uint32_t cnt = hist[b], s0 = cur[b] - cnt;
+        uint32_t r = 0;
+        for (uint32_t q = s0; q < s0 + cnt; ++q) {
+            const uint32_t kq = s.keyA[q];
+            r += (kq > kv) | ((kq == kv) & (s.idxA[q] < iv));
+        }
+        oidx[s0 + r] = iv;
+        if (oval) oval[s0 + r] = from_key(kv);
+    }
+    for (int j = m + tid; j < k; j += kTopkThreads) {
+        oidx[j] = -1;
+        if (oval) oval[j] = __uint_as_float(0xFF800000u);
+    }
+    return true;
+}
+
+__global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a)
+{
+    extern __shared__ __align__(16) uint8_t smem[];
+    __shared__ TopkShared sh;
+
+    const int tid = threadIdx.x;
+    const int row = blockIdx.x;
+    const int k = a.k;
+
+    // --- which elements of which row
+    int n = 0;
+    if (a.standalone) {
+        n = a.row_len ? a.row_len[row] : (int)a.ld;
+        n = n < 0 ? 0 : (n > a.ld ? (int)a.ld : n);
+    } else {
+        int b = -1, i = 0;
+        if (a.layout_q == LI_BSND) {
+            b = row / a.S1;
+            i = row % a.S1;
+        } else {
+            int lo = 0, hi = a.B - 1;               // last batch with q_off <= row
+            while (lo < hi) {
+                int mid = (lo + hi + 1) >> 1;
+                if (a.batches[mid].q_off <= row) lo = mid; else hi = mid - 1;
+            }
+            b = lo;
+            i = row - a.batches[b].q_off;
+        }
+        const BatchInfo bi = a.batches[b];
+        if (i >= 0 && i < bi.Sq) {
+            int nv = bi.Sk;
+            if (a.mode == 3) {
+                int lim = i + 1 + bi.Sk - bi.Sq;
+                nv = lim < 0 ? 0 : (lim < bi.Sk ? lim : bi.Sk);
+            }
+            n = nv;
+        }
+    }
+    int32_t *oidx = a.out_idx + (int64_t)row * k;
+    float *oval = a.out_val ? a.out_val + (int64_t)row * k : nullptr;
+    const int m = n < k ? n : k;
+
+    if (m == 0) {
+        for (int j = tid; j < k; j += kTopkThreads) {
+            oidx[j] = -1;
+            if (oval) oval[j] = __uint_as_float(0xFF800000u);
+        }
+        return;
+    }
+
+    TopkSmem s;
+    s.hist = reinterpret_cast<uint32_t *>(smem);
+    s.keyA = s.hist + 4096;
+    s.idxA = reinterpret_cast<int32_t *>(s.keyA + a.kmax);
+    s.keyB = reinterpret_cast<uint32_t *>(s.idxA + a.kmax);
+    s.idxB = reinterpret_cast<int32_t *>(s.keyB + a.kmax);
+    s.cache = reinterpret_cast<uint32_t *>(s.idxB + a.kmax);
+
+    if (tid == 0) {
+        sh.kmin = 0xFFFFFFFFu;
+        sh.kmax = 0u;
+    }
+    __syncthreads();
+    RowSrc src;
+    src.g = a.scores + (int64_t)row * a.ld;
+    src.c = nullptr;
+    src.n = n;
+    const int n4 = (n + 3) >> 2;
+    const bool cached = n <= a.cap;
+    uint32_t lmin = 0xFFFFFFFFu, lmax = 0u;
+    {
+        const float4 *g4 = reinterpret_cast<const float4 *>(src.g);
+        uint4 *c4 = reinterpret_cast<uint4 *>(s.cache);
+        for (int j4 = tid; j4 < n4; j4 += kTopkThreads) {
+            const float4 v = g4[j4];
+            const uint4 q = make_uint4(to_key(v.x), to_key(v.y), to_key(v.z), to_key(v.w));
+            if (cached) c4[j4] = q;
+            const uint32_t kv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (j4 * 4 + e < n) {
+                    lmin = min(lmin, kv[e]);
+                    lmax = max(lmax, kv[e]);
+                }
+        }
+    }
+    atomicMin(&sh.kmin, lmin);
+    atomicMax(&sh.kmax, lmax);
+    if (cached) src.c = s.cache;
+    __syncthreads();
+
+    if (!bucket_topk(src, n, k, m, a.kmax, s, sh, oidx, oval))
+        radix_topk(src, n, k, m, s, sh, oidx, oval);
 }
 
 }  // namespace

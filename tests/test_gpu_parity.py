@@ -161,16 +161,26 @@ def _topk_reference(rows_np, lens, k):
     return idx, val
 
 
-@pytest.mark.parametrize("ld,k,quantised", [(4096, 1024, False), (300, 64, True),
-                                            (8192, 2048, True), (40000, 2048, False),
-                                            (40000, 512, True), (64, 100, False)])
-def test_topk_stage_exact(ld, k, quantised):
+@pytest.mark.parametrize("ld,k,kind", [(4096, 1024, "normal"), (300, 64, "quarters"),
+                                       (8192, 2048, "quarters"), (40000, 2048, "normal"),
+                                       (40000, 512, "quarters"), (64, 100, "normal"),
+                                       (4096, 1024, "levels"), (16384, 2048, "levels"),
+                                       (2048, 2048, "levels"), (5000, 700, "constant")])
+def test_topk_stage_exact(ld, k, kind):
+    """Exact against a lexsort reference.  'quarters' (values on a 0.25 grid,
+    every 7th -0.0) and 'constant' rows force the radix fallback; 'levels'
+    (~7 keys per distinct value) keeps the bucket path with ties inside and
+    at the threshold bucket."""
     g = torch.Generator().manual_seed(ld + k)
     R = 12
     x = torch.randn(R, ld, generator=g)
-    if quantised:                                   # many exact ties, +0 and -0
+    if kind == "quarters":                           # many exact ties, +0 and -0
         x = torch.round(x * 4) / 4
         x[:, ::7] = -0.0
+    elif kind == "levels":
+        x = torch.randint(0, max(ld // 7, 1), (R, ld), generator=g).to(torch.float32) / 7.0 - 3.0
+    elif kind == "constant":
+        x = torch.full((R, ld), 1.5)
     lens = torch.randint(1, ld + 1, (R,), generator=g).to(torch.int32)
     lens[0] = ld
     lens[1] = min(k, ld)

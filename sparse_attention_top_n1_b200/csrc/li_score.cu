@@ -132,7 +132,7 @@ __device__ __forceinline__ void fail(PlanHeader *hdr, volatile int *abort_flag, 
 }
 
 template <int CHUNKS, int N1P, bool FP8>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(kScoreThreads, 1)
     score_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                  const ScoreArgs a)
 {
@@ -410,18 +410,6 @@ __global__ void __maxnreg__(200)
                 tc_fence_after_sync();
                 const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16) +
                                       (uint32_t)(acc * kAccCols + half * 128);
-                float v[4][32];
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    if (c < nchunks) tmem_ld32(trow + c * 32, v[c]);
-                tmem_ld_wait();
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&acc_empty[acc]);
-                if (++acc == kAccStages) {
-                    acc = 0;
-                    acc_phase ^= 1u;
-                }
                 const int t = w.tile * kTileKeys + lrow;
                 float ks = 1.f;
                 if (a.quant && t < bi.Sk) {
@@ -444,24 +432,53 @@ __global__ void __maxnreg__(200)
                 for (int q = 0; q < QPW; ++q)
 #pragma unroll
                     for (int p = 0; p < NP2; ++p) part[q][p] = 0ull;
+                // two 32-column chunks per round keep the register footprint
+                // within the 168 registers a 10-warp CTA allows
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    if (c < nchunks) {
-                        const uint4 *w4 = reinterpret_cast<const uint4 *>(myW + c * 32);
+                for (int cp = 0; cp < 2; ++cp) {
+                    if (2 * cp < nchunks) {
+                        float v[2][32];
 #pragma unroll
-                        for (int j4 = 0; j4 < 8; ++j4) {
-                            const uint4 ww = w4[j4];
-                            const int j = j4 * 4;
-                            const int q = (c * 32 + j) / N1P;      // same query for j..j+3
-                            const int p0 = (j / 2) % NP2, p1 = (j / 2 + 1) % NP2;
-                            const uint64_t w01 = pack2(__uint_as_float(ww.x), __uint_as_float(ww.y));
-                            const uint64_t w23 = pack2(__uint_as_float(ww.z), __uint_as_float(ww.w));
-                            part[q][p0] = ffma2(w01, pack2(fmaxf(v[c][j], 0.f), fmaxf(v[c][j + 1], 0.f)),
-                                                part[q][p0]);
-                            part[q][p1] = ffma2(w23, pack2(fmaxf(v[c][j + 2], 0.f), fmaxf(v[c][j + 3], 0.f)),
-                                                part[q][p1]);
+                        for (int c2 = 0; c2 < 2; ++c2)
+                            if (2 * cp + c2 < nchunks) tmem_ld32(trow + (2 * cp + c2) * 32, v[c2]);
+                        tmem_ld_wait();
+                        if (2 * cp + 2 >= nchunks) {
+                            // every column this warp needs is in registers: hand
+                            // the accumulator back to the MMA warp
+                            tc_fence_before_sync();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+                        }
+#pragma unroll
+                        for (int c2 = 0; c2 < 2; ++c2) {
+                            const int c = 2 * cp + c2;
+                            if (c < nchunks) {
+                                const uint4 *w4 = reinterpret_cast<const uint4 *>(myW + c * 32);
+#pragma unroll
+                                for (int j4 = 0; j4 < 8; ++j4) {
+                                    const uint4 ww = w4[j4];
+                                    const int j = j4 * 4;
+                                    const int q = (c * 32 + j) / N1P;   // same query for j..j+3
+                                    const int p0 = (j / 2) % NP2, p1 = (j / 2 + 1) % NP2;
+                                    const uint64_t w01 = pack2(__uint_as_float(ww.x), __uint_as_float(ww.y));
+                                    const uint64_t w23 = pack2(__uint_as_float(ww.z), __uint_as_float(ww.w));
+                                    part[q][p0] = ffma2(w01, pack2(fmaxf(v[c2][j], 0.f), fmaxf(v[c2][j + 1], 0.f)),
+                                                        part[q][p0]);
+                                    part[q][p1] = ffma2(w23, pack2(fmaxf(v[c2][j + 2], 0.f), fmaxf(v[c2][j + 3], 0.f)),
+                                                        part[q][p1]);
+                                }
+                            }
                         }
                     }
+                }
+                if (nchunks == 0) {                // nothing to read: release at once
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&acc_empty[acc]);
+                }
+                if (++acc == kAccStages) {
+                    acc = 0;
+                    acc_phase ^= 1u;
                 }
                 // visible keys only: t < nvis(i); the row keeps its visible prefix
 #pragma unroll

@@ -57,10 +57,15 @@ __device__ int32_t block_inclusive_scan(int32_t &v, int32_t *tmp)
     return total;
 }
 
+constexpr int kSmemBatches = 1024;      // batches mirrored in shared memory
+
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a)
 {
     __shared__ int32_t s_tmp[kPlanThreads / 32];
     __shared__ int32_t s_flags;
+    __shared__ int32_t s_blk_off[kSmemBatches];
+    __shared__ int2 s_len[kSmemBatches];          // (Sq, Sk)
+    const bool in_smem = a.B <= kSmemBatches;
     const int tid = threadIdx.x;
     if (tid == 0) s_flags = 0;
     __syncthreads();
@@ -121,6 +126,10 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a)
         if (b < a.B) {
             bi.blk_off = carry + incl - nblk;
             a.batches[b] = bi;
+            if (in_smem) {
+                s_blk_off[b] = bi.blk_off;
+                s_len[b] = make_int2(bi.Sq, bi.Sk);
+            }
         }
         carry += tot;
     }
@@ -143,15 +152,26 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a)
             int lo = 0, hi = a.B - 1;                  // last batch with blk_off <= g
             while (lo < hi) {
                 const int mid = (lo + hi + 1) >> 1;
-                if (a.batches[mid].blk_off <= g) lo = mid; else hi = mid - 1;
+                const int off = in_smem ? s_blk_off[mid] : a.batches[mid].blk_off;
+                if (off <= g) lo = mid; else hi = mid - 1;
             }
-            const BatchInfo bi = a.batches[lo];
-            const int32_t i0 = (g - bi.blk_off) * a.nq;
+            int32_t blk_off, Sq, Sk;
+            if (in_smem) {
+                blk_off = s_blk_off[lo];
+                Sq = s_len[lo].x;
+                Sk = s_len[lo].y;
+            } else {
+                const BatchInfo bi = a.batches[lo];
+                blk_off = bi.blk_off;
+                Sq = bi.Sq;
+                Sk = bi.Sk;
+            }
+            const int32_t i0 = (g - blk_off) * a.nq;
             int32_t i_last = i0 + a.nq;
-            if (i_last > bi.Sq) i_last = bi.Sq;
+            if (i_last > Sq) i_last = Sq;
             i_last -= 1;
-            int64_t nvis = bi.Sk;
-            if (a.mode == 3) nvis = clamp64((int64_t)i_last + 1 + bi.Sk - bi.Sq, 0, bi.Sk);
+            int64_t nvis = Sk;
+            if (a.mode == 3) nvis = clamp64((int64_t)i_last + 1 + Sk - Sq, 0, Sk);
             ntiles = (int32_t)((nvis + kTileKeys - 1) / kTileKeys);
             blk.b = lo;
             blk.i0 = i0;

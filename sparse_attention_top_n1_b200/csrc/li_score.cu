@@ -110,6 +110,13 @@ __device__ __forceinline__ uint64_t pack2(float lo, float hi)
     return r;
 }
 
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 __device__ __forceinline__ float hsum2(uint64_t r)
 {
     float lo, hi;
@@ -192,6 +199,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
+    // the prologue above overlaps the scheduler's tail; its work list is read below
+    grid_dependency_wait();
+    grid_launch_dependents();
 
     const int total = a.hdr->total_units;
     const int nblocks = a.hdr->total_blocks;
@@ -487,10 +497,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                         int nv = lim0 + q;
                         nv = nv < 0 ? 0 : (nv < bi.Sk ? nv : bi.Sk);
                         if (t < nv) {
-                            float s = 0.f;
+                            uint64_t sum2 = part[q][0];
 #pragma unroll
-                            for (int p = 0; p < NP2; ++p) s += hsum2(part[q][p]);
-                            row_ptr[(int64_t)q * a.ld + t] = s * ks;
+                            for (int p = 1; p < NP2; ++p) sum2 = fadd2(sum2, part[q][p]);
+                            row_ptr[(int64_t)q * a.ld + t] = hsum2(sum2) * ks;
                         }
                     }
                 }
@@ -512,8 +522,17 @@ cudaError_t launch_one(const ScoreArgs &a, const CUtensorMap &qmap, const CUtens
     const size_t smem = Geometry<CHUNKS>::SMEM;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kScoreThreads, smem, s>>>(qmap, kmap, a);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kScoreThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, qmap, kmap, a);
 }
 
 template <int CHUNKS, bool FP8>

@@ -22,6 +22,7 @@
 #include <cstdint>
 
 #include "li_internal.cuh"
+#include "ptx.cuh"
 
 namespace li {
 namespace {
@@ -456,6 +457,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a)
     const int tid = threadIdx.x;
     const int row = blockIdx.x;
     const int k = a.k;
+    grid_dependency_wait();             // the score rows come from the previous kernel
 
     // --- which elements of which row
     int n = 0;
@@ -557,8 +559,17 @@ cudaError_t launch_topk(const TopkArgs &a, cudaStream_t s)
                                          (int)smem);
     if (e != cudaSuccess) return e;
     if (a.rows <= 0) return cudaSuccess;
-    topk_kernel<<<a.rows, kTopkThreads, smem, s>>>(a);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.rows);
+    cfg.blockDim = dim3(kTopkThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = a.standalone ? 0 : 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, topk_kernel, a);
 }
 
 }  // namespace li

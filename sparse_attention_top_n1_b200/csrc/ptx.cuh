@@ -67,6 +67,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may be suspended in hardware for up to
+// `hint_ns` nanoseconds while the phase is incomplete (it wakes as soon as the
+// phase completes), so a waiting warp does not spin on the issue slots.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete.  Returns false when
 // `timeout_ns` elapsed first or when *abort became non-zero (another role of
 // the CTA gave up); the caller then stops its pipeline loop.
@@ -76,16 +92,30 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     if (mbar_try_wait(bar, parity))
         return true;
     const uint64_t t0 = global_timer_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity))
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 20000u))
             return true;
-        if ((it & 63u) == 0) {
-            if (abort && *abort)
-                return false;
-            if ((int64_t)(global_timer_ns() - t0) > timeout_ns)
-                return false;
-        }
+        if (abort && *abort)
+            return false;
+        if ((int64_t)(global_timer_ns() - t0) > timeout_ns)
+            return false;
     }
+}
+
+// ---------------------------------------------------------------- dependent launch
+
+// Block until every kernel this grid programmatically depends on has
+// completed and its memory is visible (a no-op without such a dependency).
+__device__ __forceinline__ void grid_dependency_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Allow the next kernel in the stream, launched with programmatic stream
+// serialization, to be scheduled before this grid has finished.
+__device__ __forceinline__ void grid_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- TMA

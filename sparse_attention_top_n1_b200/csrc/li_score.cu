@@ -138,6 +138,34 @@ __device__ __forceinline__ void fail(PlanHeader *hdr, volatile int *abort_flag, 
     *abort_flag = 1;
 }
 
+// part[q] += W[col] * ReLU(v[col]) over chunks c0, c0+1 (32 columns each) of
+// this warp's 128 columns, two columns per packed FMA.
+template <int N1P, int QPW, int NP2>
+__device__ __forceinline__ void reduce_chunks(const float (&v)[2][32], const float *myW, int c0,
+                                              int nchunks, uint64_t (&part)[QPW][NP2])
+{
+#pragma unroll
+    for (int c2 = 0; c2 < 2; ++c2) {
+        const int c = c0 + c2;
+        if (c < nchunks) {
+            const uint4 *w4 = reinterpret_cast<const uint4 *>(myW + c * 32);
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4) {
+                const uint4 ww = w4[j4];
+                const int j = j4 * 4;
+                const int q = (c * 32 + j) / N1P;          // same query for j..j+3
+                const int p0 = (j / 2) % NP2, p1 = (j / 2 + 1) % NP2;
+                const uint64_t w01 = pack2(__uint_as_float(ww.x), __uint_as_float(ww.y));
+                const uint64_t w23 = pack2(__uint_as_float(ww.z), __uint_as_float(ww.w));
+                part[q][p0] = ffma2(w01, pack2(fmaxf(v[c2][j], 0.f), fmaxf(v[c2][j + 1], 0.f)),
+                                    part[q][p0]);
+                part[q][p1] = ffma2(w23, pack2(fmaxf(v[c2][j + 2], 0.f), fmaxf(v[c2][j + 3], 0.f)),
+                                    part[q][p1]);
+            }
+        }
+    }
+}
+
 template <int CHUNKS, int N1P, bool FP8>
 __global__ void __launch_bounds__(kScoreThreads, 1)
     score_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
@@ -147,7 +175,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     constexpr int STAGES = G::STAGES;
     constexpr int NQ = 256 / N1P;                 // queries per block
     constexpr int QPW = 128 / N1P;                // queries per epilogue warp half
-    constexpr int NP2 = N1P >= 32 ? 4 : (N1P == 16 ? 2 : 1);  // packed partial sums per query
+    constexpr int NP2 = N1P >= 32 ? 2 : 1;                     // packed partial sums per query
     constexpr int INNER = FP8 ? 128 : 64;         // elements per 128-byte row chunk
 
     extern __shared__ uint8_t smem_raw[];
@@ -442,43 +470,29 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 for (int q = 0; q < QPW; ++q)
 #pragma unroll
                     for (int p = 0; p < NP2; ++p) part[q][p] = 0ull;
-                // two 32-column chunks per round keep the register footprint
-                // within the 168 registers a 10-warp CTA allows
-#pragma unroll
-                for (int cp = 0; cp < 2; ++cp) {
-                    if (2 * cp < nchunks) {
-                        float v[2][32];
-#pragma unroll
-                        for (int c2 = 0; c2 < 2; ++c2)
-                            if (2 * cp + c2 < nchunks) tmem_ld32(trow + (2 * cp + c2) * 32, v[c2]);
+                // Columns come out of TMEM in two rounds of two 32-column chunks;
+                // the second round's loads are issued before the first round is
+                // reduced, so their latency hides behind that arithmetic.
+                float v0[2][32], v1[2][32];
+                if (nchunks > 0) {
+                    tmem_ld32(trow, v0[0]);
+                    if (nchunks > 1) tmem_ld32(trow + 32, v0[1]);
+                    tmem_ld_wait();
+                    if (nchunks > 2) {
+                        tmem_ld32(trow + 64, v1[0]);
+                        if (nchunks > 3) tmem_ld32(trow + 96, v1[1]);
+                    } else {
+                        tc_fence_before_sync();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+                    }
+                    reduce_chunks<N1P, QPW, NP2>(v0, myW, 0, nchunks, part);
+                    if (nchunks > 2) {
                         tmem_ld_wait();
-                        if (2 * cp + 2 >= nchunks) {
-                            // every column this warp needs is in registers: hand
-                            // the accumulator back to the MMA warp
-                            tc_fence_before_sync();
-                            __syncwarp();
-                            if (lane == 0) mbar_arrive(&acc_empty[acc]);
-                        }
-#pragma unroll
-                        for (int c2 = 0; c2 < 2; ++c2) {
-                            const int c = 2 * cp + c2;
-                            if (c < nchunks) {
-                                const uint4 *w4 = reinterpret_cast<const uint4 *>(myW + c * 32);
-#pragma unroll
-                                for (int j4 = 0; j4 < 8; ++j4) {
-                                    const uint4 ww = w4[j4];
-                                    const int j = j4 * 4;
-                                    const int q = (c * 32 + j) / N1P;   // same query for j..j+3
-                                    const int p0 = (j / 2) % NP2, p1 = (j / 2 + 1) % NP2;
-                                    const uint64_t w01 = pack2(__uint_as_float(ww.x), __uint_as_float(ww.y));
-                                    const uint64_t w23 = pack2(__uint_as_float(ww.z), __uint_as_float(ww.w));
-                                    part[q][p0] = ffma2(w01, pack2(fmaxf(v[c2][j], 0.f), fmaxf(v[c2][j + 1], 0.f)),
-                                                        part[q][p0]);
-                                    part[q][p1] = ffma2(w23, pack2(fmaxf(v[c2][j + 2], 0.f), fmaxf(v[c2][j + 3], 0.f)),
-                                                        part[q][p1]);
-                                }
-                            }
-                        }
+                        tc_fence_before_sync();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+                        reduce_chunks<N1P, QPW, NP2>(v1, myW, 2, nchunks, part);
                     }
                 }
                 if (nchunks == 0) {                // nothing to read: release at once

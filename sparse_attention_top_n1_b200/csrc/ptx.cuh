@@ -93,7 +93,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
         return true;
     const uint64_t t0 = global_timer_ns();
     for (;;) {
-        if (mbar_try_wait_sleep(bar, parity, 20000u))
+        if (mbar_try_wait(bar, parity))
             return true;
         if (abort && *abort)
             return false;

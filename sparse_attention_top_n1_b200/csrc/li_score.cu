@@ -45,7 +45,7 @@ struct Geometry {
     static constexpr int Q_CHUNK = kQRows * kRowBytes;
     static constexpr int K_CHUNK = kTileKeys * kRowBytes;
     static constexpr int K_BYTES = K_CHUNK * CHUNKS;
-    static constexpr int W_FLOATS = kEpiWarps * kAccCols;
+    static constexpr int W_FLOATS = kEpiWarps * 128;
     static constexpr int NBARS = 2 * STAGES + 7;
     static constexpr size_t SMEM = 1024 + Q_BYTES + (size_t)STAGES * K_BYTES + W_FLOATS * 4 +
                                    NBARS * 8 + 16;
@@ -110,13 +110,6 @@ __device__ __forceinline__ uint64_t pack2(float lo, float hi)
     return r;
 }
 
-__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b)
-{
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-
 __device__ __forceinline__ float hsum2(uint64_t r)
 {
     float lo, hi;
@@ -138,28 +131,6 @@ __device__ __forceinline__ void fail(PlanHeader *hdr, volatile int *abort_flag, 
     *abort_flag = 1;
 }
 
-// Chunk c of a tile row (TMEM columns 32c .. 32c+31): part[q] += W*ReLU(v)
-// for the queries the chunk touches, two columns per packed FMA.  With
-// N1P >= 32 a query spans N1P/32 chunks and part carries over; with N1P < 32
-// a chunk holds 32/N1P whole queries.
-template <int N1P, int NP2>
-__device__ __forceinline__ void reduce_chunk(const float (&v)[32], const float *w,
-                                             uint64_t (&part)[(N1P >= 32 ? 1 : 32 / N1P)][NP2])
-{
-    const uint4 *w4 = reinterpret_cast<const uint4 *>(w);
-#pragma unroll
-    for (int j4 = 0; j4 < 8; ++j4) {
-        const uint4 ww = w4[j4];
-        const int j = j4 * 4;
-        const int q = N1P >= 32 ? 0 : j / N1P;                // same query for j..j+3
-        const int p0 = (j / 2) % NP2, p1 = (j / 2 + 1) % NP2;
-        const uint64_t w01 = pack2(__uint_as_float(ww.x), __uint_as_float(ww.y));
-        const uint64_t w23 = pack2(__uint_as_float(ww.z), __uint_as_float(ww.w));
-        part[q][p0] = ffma2(w01, pack2(fmaxf(v[j], 0.f), fmaxf(v[j + 1], 0.f)), part[q][p0]);
-        part[q][p1] = ffma2(w23, pack2(fmaxf(v[j + 2], 0.f), fmaxf(v[j + 3], 0.f)), part[q][p1]);
-    }
-}
-
 template <int CHUNKS, int N1P, bool FP8>
 __global__ void __launch_bounds__(kScoreThreads, 1)
     score_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
@@ -168,6 +139,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     using G = Geometry<CHUNKS>;
     constexpr int STAGES = G::STAGES;
     constexpr int NQ = 256 / N1P;                 // queries per block
+    constexpr int QPW = 128 / N1P;                // queries per epilogue warp half
     constexpr int NP2 = N1P >= 32 ? 4 : (N1P == 16 ? 2 : 1);  // packed partial sums per query
     constexpr int INNER = FP8 ? 128 : 64;         // elements per 128-byte row chunk
 
@@ -199,7 +171,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         mbar_init(q_empty, 1);
         for (int s = 0; s < kAccStages; ++s) {
             mbar_init(&acc_full[s], 1);
-            mbar_init(&acc_empty[s], kEpiWarps / kAccStages);
+            mbar_init(&acc_empty[s], kEpiWarps);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -383,40 +355,41 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        // Warps 2-5 reduce the tiles of accumulator 0 and warps 6-9 those of
-        // accumulator 1, so the two epilogue warps sharing an SM sub-partition
-        // work one tile apart and hide each other's TMEM and memory latency.
-        // A thread owns key row `lrow` of its tile and all 256 columns
-        // (NQ queries x N1P heads); it reads them from TMEM in rounds of 64
-        // columns, the next round's loads in flight while the current round
-        // is reduced (sum_h W*ReLU(logit), two columns per packed FMA) and its
-        // queries' scores are written.
+        // Each thread owns key row `lrow` of the tile and the 128 columns of
+        // its warp half: QPW queries x N1P heads.  Per tile it loads those
+        // columns from TMEM in one go, hands the accumulator back to the MMA
+        // warp, then reduces sum_h W*ReLU(logit) with packed fp32 FMAs.
         const int ew = warp - 2;                   // 0..7
         const int quarter = warp & 3;              // TMEM lanes this warp may access
-        const int my_acc = ew >> 2;                // accumulator stage this warp serves
+        const int half = ew >> 2;                  // which 128 of the 256 columns
         const int lrow = quarter * 32 + lane;      // key row within the tile
-        float *myW = sW + ew * kAccCols;
+        float *myW = sW + ew * 128;
         if (w_begin < w_end && nblocks > 0) {
             Walker w{a.blocks, nblocks, 0, 0, 0, 0, 0};
             w.init(w_begin, w_end);
-            int prev_qb = -1, nchunks = 0, nrows = 0, local = 0;
+            int acc = 0, prev_qb = -1, nchunks = 0;
             uint32_t acc_phase = 0;
             BlockInfo blk{};
             BatchInfo bi{};
-            float *row_ptr = nullptr;              // score row of the block's first query
-            int lim0 = 0;                          // visible-key limit of that query
-            for (; w.valid(); w.next(), ++local) {
+            float *row_ptr = nullptr;              // score row of this half's first query
+            int lim0 = 0, nq_valid = 0;            // visible limit of that query; valid queries
+            for (; w.valid(); w.next()) {
                 if (w.qb != prev_qb) {
                     blk = a.blocks[w.qb];
                     bi = a.batches[blk.b];
-                    nrows = bi.Sq - blk.i0;
+                    int nrows = bi.Sq - blk.i0;
                     nrows = nrows > NQ ? NQ : nrows;
-                    nchunks = (nrows * N1P + 31) / 32;
-                    row_ptr = a.scores + (int64_t)(bi.row0 + blk.i0) * a.ld;
-                    lim0 = a.mode == 3 ? blk.i0 + 1 + bi.Sk - bi.Sq : bi.Sk;
+                    int mine = nrows - half * QPW;     // valid queries of this half
+                    mine = mine < 0 ? 0 : (mine > QPW ? QPW : mine);
+                    nq_valid = mine;
+                    nchunks = (mine * N1P + 31) / 32;
+                    const int i_first = blk.i0 + half * QPW;
+                    row_ptr = a.scores + (int64_t)(bi.row0 + i_first) * a.ld;
+                    lim0 = a.mode == 3 ? i_first + 1 + bi.Sk - bi.Sq : bi.Sk;
                     __syncwarp();
-                    for (int j = lane; j < kAccCols; j += 32) {
-                        const int q = j / N1P, h = j % N1P;
+                    for (int j = lane; j < 128; j += 32) {
+                        const int col = half * 128 + j;
+                        const int q = col / N1P, h = col % N1P;
                         const int i = blk.i0 + q;
                         float wv = 0.f;
                         if (h < a.N1 && i < bi.Sq) {
@@ -433,15 +406,13 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                     __syncwarp();
                     prev_qb = w.qb;
                 }
-                if ((local & 1) != my_acc) continue;            // the other warp's tile
-                if (!mbar_wait_bounded(&acc_full[my_acc], acc_phase, abort_flag, a.timeout_ns)) {
+                if (!mbar_wait_bounded(&acc_full[acc], acc_phase, abort_flag, a.timeout_ns)) {
                     fail(a.hdr, abort_flag, LI_DEV_TIMEOUT);
                     break;
                 }
-                acc_phase ^= 1u;
                 tc_fence_after_sync();
                 const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16) +
-                                      (uint32_t)(my_acc * kAccCols);
+                                      (uint32_t)(acc * kAccCols + half * 128);
                 const int t = w.tile * kTileKeys + lrow;
                 float ks = 1.f;
                 if (a.quant && t < bi.Sk) {
@@ -459,52 +430,72 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                         if (ks < 0.f) atomicOr(&a.hdr->status, LI_DEV_NEG_SCALE);
                     }
                 }
-                constexpr int QPC = N1P >= 32 ? 1 : 32 / N1P;   // queries per chunk
-                constexpr int CPQ = N1P >= 32 ? N1P / 32 : 1;   // chunks per query
-                float vb[2][32];                               // two chunks in flight
-                uint64_t part[QPC][NP2];
-                if (nchunks > 0) tmem_ld32(trow, vb[0]);
+                uint64_t part[QPW][NP2];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    if (c < nchunks) {
+                for (int q = 0; q < QPW; ++q)
+#pragma unroll
+                    for (int p = 0; p < NP2; ++p) part[q][p] = 0ull;
+                // two 32-column chunks per round keep the register footprint
+                // within the 168 registers a 10-warp CTA allows
+#pragma unroll
+                for (int cp = 0; cp < 2; ++cp) {
+                    if (2 * cp < nchunks) {
+                        float v[2][32];
+#pragma unroll
+                        for (int c2 = 0; c2 < 2; ++c2)
+                            if (2 * cp + c2 < nchunks) tmem_ld32(trow + (2 * cp + c2) * 32, v[c2]);
                         tmem_ld_wait();
-                        if (c + 1 < nchunks) {
-                            tmem_ld32(trow + (c + 1) * 32, vb[(c + 1) & 1]);
-                        } else {
-                            // every column is in registers: hand the accumulator back
+                        if (2 * cp + 2 >= nchunks) {
+                            // every column this warp needs is in registers: hand
+                            // the accumulator back to the MMA warp
                             tc_fence_before_sync();
                             __syncwarp();
-                            if (lane == 0) mbar_arrive(&acc_empty[my_acc]);
+                            if (lane == 0) mbar_arrive(&acc_empty[acc]);
                         }
-                        if (c % CPQ == 0) {
 #pragma unroll
-                            for (int q = 0; q < QPC; ++q)
+                        for (int c2 = 0; c2 < 2; ++c2) {
+                            const int c = 2 * cp + c2;
+                            if (c < nchunks) {
+                                const uint4 *w4 = reinterpret_cast<const uint4 *>(myW + c * 32);
 #pragma unroll
-                                for (int p = 0; p < NP2; ++p) part[q][p] = 0ull;
-                        }
-                        reduce_chunk<N1P, NP2>(vb[c & 1], myW + c * 32, part);
-                        if ((c + 1) % CPQ == 0) {
-#pragma unroll
-                            for (int q = 0; q < QPC; ++q) {
-                                const int qi = (c / CPQ) * QPC + q;   // query within the block
-                                if (qi < nrows) {
-                                    int nv = lim0 + qi;
-                                    nv = nv < 0 ? 0 : (nv < bi.Sk ? nv : bi.Sk);
-                                    if (t < nv) {
-                                        uint64_t sum2 = part[q][0];
-#pragma unroll
-                                        for (int p = 1; p < NP2; ++p) sum2 = fadd2(sum2, part[q][p]);
-                                        row_ptr[(int64_t)qi * a.ld + t] = hsum2(sum2) * ks;
-                                    }
+                                for (int j4 = 0; j4 < 8; ++j4) {
+                                    const uint4 ww = w4[j4];
+                                    const int j = j4 * 4;
+                                    const int q = (c * 32 + j) / N1P;   // same query for j..j+3
+                                    const int p0 = (j / 2) % NP2, p1 = (j / 2 + 1) % NP2;
+                                    const uint64_t w01 = pack2(__uint_as_float(ww.x), __uint_as_float(ww.y));
+                                    const uint64_t w23 = pack2(__uint_as_float(ww.z), __uint_as_float(ww.w));
+                                    part[q][p0] = ffma2(w01, pack2(fmaxf(v[c2][j], 0.f), fmaxf(v[c2][j + 1], 0.f)),
+                                                        part[q][p0]);
+                                    part[q][p1] = ffma2(w23, pack2(fmaxf(v[c2][j + 2], 0.f), fmaxf(v[c2][j + 3], 0.f)),
+                                                        part[q][p1]);
                                 }
                             }
                         }
                     }
                 }
-                if (nchunks == 0) {                 // nothing to read: release at once
+                if (nchunks == 0) {                // nothing to read: release at once
                     tc_fence_before_sync();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&acc_empty[my_acc]);
+                    if (lane == 0) mbar_arrive(&acc_empty[acc]);
+                }
+                if (++acc == kAccStages) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+                // visible keys only: t < nvis(i); the row keeps its visible prefix
+#pragma unroll
+                for (int q = 0; q < QPW; ++q) {
+                    if (q < nq_valid) {
+                        int nv = lim0 + q;
+                        nv = nv < 0 ? 0 : (nv < bi.Sk ? nv : bi.Sk);
+                        if (t < nv) {
+                            float s = 0.f;
+#pragma unroll
+                            for (int p = 0; p < NP2; ++p) s += hsum2(part[q][p]);
+                            row_ptr[(int64_t)q * a.ld + t] = s * ks;
+                        }
+                    }
                 }
             }
         }

@@ -162,6 +162,40 @@ LI_API li_status li_quant_indexer(const li_params *p, const void *query, const v
 LI_API li_status li_topk(const float *scores, int64_t ld, const int32_t *row_len, int32_t rows,
                   int32_t k, int32_t *sparse_indices, float *sparse_values, void *stream);
 
+/*
+ * li_indexer for callers that cannot hand the library any device memory of
+ * their own.  The pages have no counterpart to it; it is an addition of this
+ * library.
+ *
+ * Some callers cannot allocate device memory: an operator interface that
+ * passes a kernel only its input and output tensors and has no workspace
+ * mechanism, or a serving loop that keeps cudaMalloc off its hot path (the
+ * call can synchronise the device and fragment a pre-reserved pool).  This
+ * entry point takes the same arguments as li_indexer minus the workspace and
+ * uses instead a scratch array of LI_NOALLOC_SCRATCH_BYTES compiled into the
+ * library: every GPU that loads the library holds that memory until the
+ * process exits.  It calls no allocator itself.
+ *
+ *   - Problems whose li_workspace_size exceeds LI_NOALLOC_SCRATCH_BYTES are
+ *     rejected with LI_ERR_WORKSPACE before anything is launched; use
+ *     li_indexer with a workspace for them.
+ *   - The first call on a device looks up that device's copy of the array
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls on a device share the one array and it keeps the contents of
+ *     the last call.  Nothing in it has to start at zero (each call's
+ *     scheduler overwrites the status and tables, and every score is written
+ *     before it is read), but calls that may overlap on the GPU -- concurrent
+ *     streams, or threads launching at the same time -- race on it.
+ *   - The device status word of these calls sits in the library's scratch
+ *     and is not exposed; use li_indexer with a workspace when the LI_DEV_*
+ *     bits are needed.
+ */
+#define LI_NOALLOC_SCRATCH_BYTES (32u << 20)
+LI_API li_status li_indexer_noalloc(const li_params *p, const void *query, const void *key,
+                                    const void *weights, const int32_t *act_seq_q,
+                                    const int32_t *act_seq_k, const int32_t *block_table,
+                                    int32_t *sparse_indices, float *sparse_values, void *stream);
+
 /* Thread-local message describing the last non-OK status. */
 LI_API const char *li_last_error(void);
 

@@ -30,7 +30,7 @@ INT64_MAX = (1 << 63) - 1
 
 EXPORTS = ("li_output_shape", "li_workspace_size", "li_indexer", "li_quant_indexer", "li_topk",
            "li_last_error", "li_read_device_status", "li_selftest_bounded_wait",
-           "li_last_launch_count", "li_set_profile_events")
+           "li_last_launch_count", "li_set_profile_events", "li_indexer_noalloc")
 
 
 class LiError(RuntimeError):
@@ -80,6 +80,7 @@ def lib() -> ctypes.CDLL:
             "li_selftest_bounded_wait": (ctypes.c_int, [vp, i64, vp]),
             "li_last_launch_count": (i32, []),
             "li_set_profile_events": (None, [ctypes.POINTER(ctypes.c_void_p), i32]),
+            "li_indexer_noalloc": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -171,6 +172,15 @@ def li_quant_indexer(params, query, key, weights, q_scale, k_scale, act_seq_q, a
 def li_topk(scores, ld, row_len, rows, k, sparse_indices, sparse_values=None, stream=None):
     _check(lib().li_topk(_ptr(scores), ld, _ptr(row_len), rows, k, _ptr(sparse_indices),
                          _ptr(sparse_values), _stream(stream)))
+
+
+def li_indexer_noalloc(params, query, key, weights, act_seq_q, act_seq_k, block_table,
+                       sparse_indices, sparse_values, stream=None):
+    """li_indexer with the library's built-in scratch instead of a workspace
+    (see include/li.h: for callers that cannot allocate device memory)."""
+    _check(lib().li_indexer_noalloc(ctypes.byref(params), _ptr(query), _ptr(key), _ptr(weights),
+                                    _ptr(act_seq_q), _ptr(act_seq_k), _ptr(block_table),
+                                    _ptr(sparse_indices), _ptr(sparse_values), _stream(stream)))
 
 
 def li_read_device_status(workspace, stream=None) -> int:

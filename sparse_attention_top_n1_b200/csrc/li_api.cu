@@ -366,6 +366,12 @@ li_status run(const li_params *pp, bool quant, const void *query, const void *ke
 
 }  // namespace
 
+namespace li {
+// Record `msg` as the thread's last error and return `s` (for the other
+// translation units of the library).
+li_status report_error(li_status s, const char *msg) { return fail(s, "%s", msg); }
+}  // namespace li
+
 extern "C" {
 
 li_status li_output_shape(const li_params *p, int64_t out_dims[4], int32_t *ndim)

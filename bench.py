@@ -51,12 +51,22 @@ WORKLOAD_DESC = {
 RETURN_VALUE = {"tiny": 1, "cfg2": 1, "dsa_prefill": 1, "paged_decode": 0, "quant_varlen": 0}
 
 
-def make_workload(name):
+SEEDS = {"tiny": 0, "cfg2": 1, "dsa_prefill": 2, "paged_decode": 3, "quant_varlen": 4}
+
+
+def make_workload(name, rank=0):
+    """The named workload; rank r > 0 draws an independent problem of the same
+    shape (seed offset by r), as weak scaling over independent problems."""
     import synth
     fn = synth.WORKLOADS[name]
     if name in ("tiny",):
-        return fn()
-    return fn(return_value=RETURN_VALUE[name])
+        return fn(seed=SEEDS[name] + rank)
+    return fn(seed=SEEDS[name] + rank, return_value=RETURN_VALUE[name])
+
+
+def job_value(rows_per_rank, steps, world, max_total_ms):
+    """Whole-job queries/s: every rank's rows over the slowest rank's time."""
+    return world * rows_per_rank * steps / (max_total_ms * 1e-3)
 
 
 def work_counts(p, inp):
@@ -190,12 +200,13 @@ def dist_setup():
     return ws, rank, local
 
 
-def allreduce_max(x):
+def allreduce_max(x, device="cuda"):
+    """Max of a host float over all ranks (timing only; no data-path use)."""
     import torch
     import torch.distributed as dist
     if not dist.is_initialized():
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -306,7 +317,7 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
 
-    p, inp = make_workload(args.workload)
+    p, inp = make_workload(args.workload, rank)
     counts = work_counts(p, inp)
     d = {k: v.to(dev) for k, v in inp.items()}
     pr = li.make_params(p)
@@ -345,35 +356,52 @@ def main():
 
     K = args.steps
     mk = lambda: torch.cuda.Event(enable_timing=True)
-    starts = [mk() for _ in range(K)]
-    ends = [mk() for _ in range(K)]
-    prof = [[mk() for _ in range(4)] for _ in range(K)]
-    for e in [x for row in prof for x in row]:      # torch creates events lazily
-        e.record()
-    torch.cuda.synchronize()
-    barrier()
-    torch.cuda.synchronize()
-    launches = 0
-    for s in range(K):
-        flush.zero_()
-        if not args.no_stage_events:
-            li.li_set_profile_events(prof[s])
-        starts[s].record()
-        call(*args_dev)
-        ends[s].record()
-        launches += li.li_last_launch_count()
-    li.li_set_profile_events(None)
-    torch.cuda.synchronize()
-    barrier()
-    clk = clocks.stop()
-    step_ms = [starts[s].elapsed_time(ends[s]) for s in range(K)]
-    total_ms = allreduce_max(sum(step_ms))
+
+    def timed_steps(stage_events):
+        """K steps, L2 flushed before each outside the timed interval.  With
+        stage_events, the library records per-kernel events inside each step
+        (which keeps the kernels from overlapping their launch with the
+        previous kernel's tail, so the step itself gets a little slower)."""
+        starts = [mk() for _ in range(K)]
+        ends = [mk() for _ in range(K)]
+        prof = [[mk() for _ in range(4)] for _ in range(K)]
+        for e in [x for row in prof for x in row]:      # torch creates events lazily
+            e.record()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        nlaunch = 0
+        for s in range(K):
+            flush.zero_()
+            if stage_events:
+                li.li_set_profile_events(prof[s])
+            starts[s].record()
+            call(*args_dev)
+            ends[s].record()
+            nlaunch += li.li_last_launch_count()
+        li.li_set_profile_events(None)
+        torch.cuda.synchronize()
+        barrier()
+        step_ms = [starts[s].elapsed_time(ends[s]) for s in range(K)]
+        stage = {"scheduler": [], "score": [], "topk": []}
+        if stage_events:
+            for s in range(K):
+                e = prof[s]
+                stage["scheduler"].append(e[0].elapsed_time(e[1]))
+                stage["score"].append(e[1].elapsed_time(e[2]))
+                stage["topk"].append(e[2].elapsed_time(e[3]))
+        return sum(step_ms), stage, nlaunch
+
+    # timed region 1: the job value, nothing between the kernels
+    own_ms, _, launches = timed_steps(False)
+    total_ms = allreduce_max(own_ms)
+    # timed region 2: the same steps with per-kernel events, for the roofline
+    staged_ms = 0.0
     stage = {"scheduler": [], "score": [], "topk": []}
-    for s in range(K if not args.no_stage_events else 0):
-        e = prof[s]
-        stage["scheduler"].append(e[0].elapsed_time(e[1]))
-        stage["score"].append(e[1].elapsed_time(e[2]))
-        stage["topk"].append(e[2].elapsed_time(e[3]))
+    if not args.no_stage_events:
+        own_staged, stage, _ = timed_steps(True)
+        staged_ms = allreduce_max(own_staged)
+    clk = clocks.stop()
     avg = {k: (sum(v) / len(v) if v else float("nan")) for k, v in stage.items()}
 
     peaks, peak_src = load_peaks()
@@ -397,7 +425,7 @@ def main():
     roof["kernel"] = dom
 
     n = ws
-    value = n * p.rows * K / (total_ms * 1e-3)
+    value = job_value(p.rows, K, n, total_ms)
     eff_tflops = n * counts["flops"] * K / (total_ms * 1e-3) / 1e12
     whole_frac = max(counts["flops"] / (tensor_peak * 1e12),
                      counts["compulsory_bytes"] / (peaks["hbm_gbs"] * 1e9)) / (total_ms * 1e-3 / K)
@@ -445,6 +473,7 @@ def main():
                    "return_value": p.return_value,
                    "l2": "flushed (256 MiB write) before every timed step",
                    "parallelism": "independent replica per GPU" if n > 1 else "1 GPU"},
+        "ms_per_step_with_stage_events": (staged_ms / K) if staged_ms else None,
         "effective_tflops": eff_tflops,
         "whole_call_roofline_frac": whole_frac,
         "roofline": roof,

@@ -1,0 +1,72 @@
+"""The N > 1 path of bench.py, on CPU with the gloo backend (world size 2).
+
+Under torchrun every rank runs an independent problem of the same shape (weak
+scaling over independent query rows: the indexer has no data-path exchange),
+the job time is the max over ranks and rank 0 reports every rank's rows over
+that time.  These tests run two real processes to check the reduction, the
+per-rank problems and the reference arm's rank handling.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import os
+import socket
+
+import torch
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    own_ms = [3.0, 7.5][rank]
+    mx = bench.allreduce_max(own_ms, device="cpu")
+    bench.barrier()
+    p, inp = bench.make_workload("tiny", rank)
+    q.put((rank, mx, p.rows, float(inp["query"].float().sum())))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_reduce_max_and_draw_independent_problems():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for pr in procs:
+        pr.start()
+    out = sorted(q.get(timeout=120) for _ in range(2))
+    for pr in procs:
+        pr.join(timeout=60)
+        assert pr.exitcode == 0
+    (r0, mx0, rows0, s0), (r1, mx1, rows1, s1) = out
+    assert mx0 == mx1 == 7.5                 # the slowest rank's time
+    assert rows0 == rows1                    # same shape on every rank
+    assert s0 != s1                          # but independent data
+    # whole-job value: all ranks' rows over the slowest rank's time
+    assert abs(bench.job_value(rows0, 10, 2, 7.5) - 2 * rows0 * 10 / 7.5e-3) < 1e-6
+
+
+def test_reference_arm_other_ranks_exit_without_work(capsys):
+    args = argparse.Namespace(workload="tiny", steps=1, warmup=3)
+    assert bench.run_reference(args, 2, 1) == 0
+    assert capsys.readouterr().out == ""
+
+
+def test_single_process_reduction_is_identity():
+    assert bench.allreduce_max(4.25, device="cpu") == 4.25
+    assert not torch.distributed.is_initialized()

@@ -210,13 +210,13 @@ bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 int topk_cap(int64_t ld, int k, int kmax)
 {
-    // shared memory budget of ~112 KB keeps two Top-k CTAs per SM
-    const int64_t budget = 112 * 1024 - 4096 * 4 - (int64_t)kmax * 16;
-    int64_t cap = budget / 4;
+    // rows of up to 16384 keys are cached in shared memory (at most ~100 KB
+    // per CTA, two CTAs per SM); longer rows stream from L2
+    int64_t cap = 16384;
     if (cap > ld) cap = ld;
-    if (cap < 0) cap = 0;
     (void)k;
-    return (int)(cap & ~int64_t(3));
+    (void)kmax;
+    return (int)((cap + 3) & ~int64_t(3));
 }
 
 li_status run(const li_params *pp, bool quant, const void *query, const void *key,

@@ -28,7 +28,8 @@ namespace li {
 namespace {
 
 constexpr int kWarps = kTopkThreads / 32;
-constexpr int kSortMaxRounds = 4;     // kmax <= 2048: 128 elements per warp
+constexpr int kSortMaxRounds = 2048 / (kWarps * 32);   // rounds of 32 per warp for kmax <= 2048
+static_assert(kWarps * 256 <= 4096, "per-warp radix counters must fit the 4096-word histogram");
 
 __device__ __forceinline__ uint32_t to_key(float f)
 {
@@ -99,7 +100,9 @@ struct TopkSmem {
     uint32_t *hist;     // 4096 words: radix histograms, or bucket counts + cursors
     uint32_t *keyA;     // kmax selected keys
     int32_t *idxA;
-    uint32_t *keyB;     // kmax: radix ping-pong buffer / bucket threshold-bin candidates
+    uint32_t *candK;    // threshold-bucket candidates of the bucket path
+    int32_t *candI;
+    uint32_t *keyB;     // kmax: radix ping-pong buffer (aliases the cache, dead by then)
     int32_t *idxB;
     uint32_t *cache;    // the row as keys, when it fits
 };
@@ -273,16 +276,23 @@ __device__ void radix_topk(const RowSrc &src, int n, int k, int m, const TopkSme
                 __syncwarp();
             }
             __syncthreads();
-            // exclusive scan over (digit major, warp minor): thread t owns digit t>>1,
-            // warps (t&1)*8 .. +8
-            const int d0 = tid >> 1, w0 = (tid & 1) * 8;
+            // exclusive scan over (digit major, warp minor): thread t owns the
+            // 8 consecutive counters 8t .. 8t+7 of that order
             uint32_t own[8], sum = 0;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) { own[j] = hist[(w0 + j) * 256 + d0]; sum += own[j]; }
+            for (int j = 0; j < 8; ++j) {
+                const int c = tid * 8 + j, d = c / kWarps, wi = c % kWarps;
+                own[j] = hist[wi * 256 + d];
+                sum += own[j];
+            }
             uint32_t tot;
             uint32_t off = block_exclusive_scan<uint32_t>(sum, s_tmp32, tot);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) { hist[(w0 + j) * 256 + d0] = off; off += own[j]; }
+            for (int j = 0; j < 8; ++j) {
+                const int c = tid * 8 + j, d = c / kWarps, wi = c % kWarps;
+                hist[wi * 256 + d] = off;
+                off += own[j];
+            }
             __syncthreads();
 #pragma unroll
             for (int r = 0; r < kSortMaxRounds; ++r) {
@@ -388,7 +398,7 @@ __device__ bool bucket_topk(const RowSrc &src, int n, int k, int m, int kmax, co
     }
     if (lmax) atomicMax(&sh.maxbin, lmax);
     __syncthreads();
-    if (sh.maxbin > (uint32_t)kBinLimit || cstar > (uint32_t)min(kCandLimit, kmax)) return false;
+    if (sh.maxbin > (uint32_t)kBinLimit || cstar > (uint32_t)kCandLimit) return false;
 
     // scatter: selected buckets into keyA/idxA at their bucket slots, the
     // threshold bucket into keyB/idxB
@@ -406,8 +416,8 @@ __device__ bool bucket_topk(const RowSrc &src, int n, int k, int m, int kmax, co
                 s.idxA[pos] = j;
             } else if (b == bstar) {
                 const uint32_t pos = atomicAdd(&cur[b], 1u) - above;
-                s.keyB[pos] = kv[e];
-                s.idxB[pos] = j;
+                s.candK[pos] = kv[e];
+                s.candI[pos] = j;
             }
         }
     }
@@ -416,12 +426,12 @@ __device__ bool bucket_topk(const RowSrc &src, int n, int k, int m, int kmax, co
     // the threshold bucket: keep the `need` best, ranked among themselves
     const uint32_t need = (uint32_t)m - above;
     for (uint32_t e = tid; e < cstar; e += kTopkThreads) {
-        const uint32_t kv = s.keyB[e];
-        const int32_t iv = s.idxB[e];
+        const uint32_t kv = s.candK[e];
+        const int32_t iv = s.candI[e];
         uint32_t r = 0;
         for (uint32_t q = 0; q < cstar; ++q) {
-            const uint32_t kq = s.keyB[q];
-            r += (kq > kv) | ((kq == kv) & (s.idxB[q] < iv));
+            const uint32_t kq = s.candK[q];
+            r += (kq > kv) | ((kq == kv) & (s.candI[q] < iv));
         }
         if (r < need) {
             oidx[above + r] = iv;
@@ -504,9 +514,11 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a)
     s.hist = reinterpret_cast<uint32_t *>(smem);
     s.keyA = s.hist + 4096;
     s.idxA = reinterpret_cast<int32_t *>(s.keyA + a.kmax);
-    s.keyB = reinterpret_cast<uint32_t *>(s.idxA + a.kmax);
-    s.idxB = reinterpret_cast<int32_t *>(s.keyB + a.kmax);
-    s.cache = reinterpret_cast<uint32_t *>(s.idxB + a.kmax);
+    s.candK = reinterpret_cast<uint32_t *>(s.idxA + a.kmax);
+    s.candI = reinterpret_cast<int32_t *>(s.candK + kCandLimit);
+    s.cache = reinterpret_cast<uint32_t *>(s.candI + kCandLimit);
+    s.keyB = s.cache;                                   // used only after the cache is dead
+    s.idxB = reinterpret_cast<int32_t *>(s.cache + a.kmax);
 
     if (tid == 0) {
         sh.kmin = 0xFFFFFFFFu;
@@ -549,7 +561,9 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a)
 
 size_t topk_smem_bytes(int cap, int kmax)
 {
-    return (size_t)4096 * 4 + (size_t)kmax * 16 + (size_t)((cap + 3) & ~3) * 4;
+    const size_t cache = (size_t)((cap + 3) & ~3) * 4, pingpong = (size_t)kmax * 8;
+    return (size_t)4096 * 4 + (size_t)kmax * 8 + (size_t)kCandLimit * 8 +
+           (cache > pingpong ? cache : pingpong);
 }
 
 cudaError_t launch_topk(const TopkArgs &a, cudaStream_t s)

@@ -186,8 +186,8 @@ li_status encode(CUtensorMap *m, int es, const void *base, int rank, const uint6
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(LI_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-    cuuint64_t d[3], s[2];
-    cuuint32_t b[3], e[3] = {1, 1, 1};
+    cuuint64_t d[4], s[3];
+    cuuint32_t b[4], e[4] = {1, 1, 1, 1};
     for (int i = 0; i < rank; ++i) { d[i] = dims[i]; b[i] = box[i]; }
     for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
     CUresult r = fn(m, es == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16,
@@ -260,10 +260,21 @@ li_status run(const li_params *pp, bool quant, const void *query, const void *ke
     BlockInfo *blocks = reinterpret_cast<BlockInfo *>(ws + w.blocks);
     float *scores = reinterpret_cast<float *>(ws + w.scores);
 
-    // query: 2-D [rows*N1, D]
+    // Tensor maps.  With 256-byte operand rows (bf16/fp16, D = 128) a row is
+    // two 128-byte swizzle chunks; an outer map dimension of extent 2 and
+    // stride 128 B walks them, so one copy fills both chunk planes of a tile
+    // ([chunk][row][128 B] in shared memory).  Otherwise one copy per chunk.
     CUtensorMap qmap, kmap;
     const int q_box_rows = (p.N1 == t.n1p) ? 256 : p.N1;
-    {
+    const bool two = t.chunks == 2;
+    int q_single = 0, k_single = 0;
+    if (two && q_box_rows == 256) {
+        const uint64_t dims[3] = {(uint64_t)inner, (uint64_t)(w.rows * p.N1), 2};
+        const uint64_t strides[2] = {(uint64_t)p.D * es, 128};
+        const uint32_t box[3] = {(uint32_t)inner, 256, 2};
+        if ((st = encode(&qmap, es, query, 3, dims, strides, box, "query")) != LI_OK) return st;
+        q_single = 1;
+    } else {
         const uint64_t dims[2] = {(uint64_t)p.D, (uint64_t)(w.rows * p.N1)};
         const uint64_t strides[1] = {(uint64_t)p.D * es};
         const uint32_t box[2] = {(uint32_t)inner, (uint32_t)q_box_rows};
@@ -272,20 +283,36 @@ li_status run(const li_params *pp, bool quant, const void *query, const void *ke
     int pa_box_rows = 0;
     if (p.layout_k != LI_PA_BSND) {
         const int64_t krows = p.layout_k == LI_BSND ? (int64_t)p.B * p.S2 : p.T2;
-        const uint64_t dims[2] = {(uint64_t)p.D, (uint64_t)krows};
-        const uint64_t strides[1] = {(uint64_t)p.D * es};
-        const uint32_t box[2] = {(uint32_t)inner, (uint32_t)kTileKeys};
-        if ((st = encode(&kmap, es, key, 2, dims, strides, box, "key")) != LI_OK) return st;
+        if (two) {
+            const uint64_t dims[3] = {(uint64_t)inner, (uint64_t)krows, 2};
+            const uint64_t strides[2] = {(uint64_t)p.D * es, 128};
+            const uint32_t box[3] = {(uint32_t)inner, (uint32_t)kTileKeys, 2};
+            if ((st = encode(&kmap, es, key, 3, dims, strides, box, "key")) != LI_OK) return st;
+            k_single = 1;
+        } else {
+            const uint64_t dims[2] = {(uint64_t)p.D, (uint64_t)krows};
+            const uint64_t strides[1] = {(uint64_t)p.D * es};
+            const uint32_t box[2] = {(uint32_t)inner, (uint32_t)kTileKeys};
+            if ((st = encode(&kmap, es, key, 2, dims, strides, box, "key")) != LI_OK) return st;
+        }
     } else {
         int g = 128;
         while (p.block_size % g) g >>= 1;               // gcd(block_size, 128) >= 16
         pa_box_rows = g;
         const int64_t stride = p.key_block_stride ? p.key_block_stride
                                                   : (int64_t)p.block_size * p.N2 * p.D;
-        const uint64_t dims[3] = {(uint64_t)p.D, (uint64_t)p.block_size, (uint64_t)p.num_blocks};
-        const uint64_t strides[2] = {(uint64_t)p.D * p.N2 * es, (uint64_t)stride * es};
-        const uint32_t box[3] = {(uint32_t)inner, (uint32_t)g, 1};
-        if ((st = encode(&kmap, es, key, 3, dims, strides, box, "paged key")) != LI_OK) return st;
+        if (two && g == kTileKeys) {
+            const uint64_t dims[4] = {(uint64_t)inner, (uint64_t)p.block_size, 2, (uint64_t)p.num_blocks};
+            const uint64_t strides[3] = {(uint64_t)p.D * p.N2 * es, 128, (uint64_t)stride * es};
+            const uint32_t box[4] = {(uint32_t)inner, (uint32_t)g, 2, 1};
+            if ((st = encode(&kmap, es, key, 4, dims, strides, box, "paged key")) != LI_OK) return st;
+            k_single = 1;
+        } else {
+            const uint64_t dims[3] = {(uint64_t)p.D, (uint64_t)p.block_size, (uint64_t)p.num_blocks};
+            const uint64_t strides[2] = {(uint64_t)p.D * p.N2 * es, (uint64_t)stride * es};
+            const uint32_t box[3] = {(uint32_t)inner, (uint32_t)g, 1};
+            if ((st = encode(&kmap, es, key, 3, dims, strides, box, "paged key")) != LI_OK) return st;
+        }
     }
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -333,6 +360,8 @@ li_status run(const li_params *pp, bool quant, const void *query, const void *ke
     sa.num_blocks = p.num_blocks;
     sa.pa_box_rows = pa_box_rows;
     sa.q_box_rows = q_box_rows;
+    sa.q_single = q_single;
+    sa.k_single = k_single;
     const uint32_t fmt = quant ? 0u : (p.dtype_qk == LI_BF16 ? 1u : 0u);
     sa.idesc_base = make_idesc(fmt, fmt, 128, 0);
     sa.timeout_ns = kDefaultTimeoutNs;

@@ -93,6 +93,7 @@ struct ScoreArgs {
     int32_t dtype_w;
     int32_t block_size, max_blocks_per_seq, num_blocks, pa_box_rows;
     int32_t q_box_rows;         // rows per Q TMA box: n1p*nq (packed) or N1 (per query)
+    int32_t q_single, k_single; // one copy covers both 128-byte chunks (3-D / 4-D maps)
     uint32_t idesc_base;        // instruction descriptor without N
     int64_t timeout_ns;
 };

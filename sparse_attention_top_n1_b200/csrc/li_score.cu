@@ -47,8 +47,9 @@ struct Geometry {
     static constexpr int K_BYTES = K_CHUNK * CHUNKS;
     static constexpr int W_FLOATS = kEpiWarps * 128;
     static constexpr int NBARS = 2 * STAGES + 7;
+    static constexpr int TABLE = 1024;         // block_table entries of one batch staged in smem
     static constexpr size_t SMEM = 1024 + Q_BYTES + (size_t)STAGES * K_BYTES + W_FLOATS * 4 +
-                                   NBARS * 8 + 16;
+                                   TABLE * 4 + NBARS * 8 + 16;
 };
 
 // Walks this CTA's share [w0, w1) of the weighted work list.  A block of n
@@ -149,7 +150,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     uint8_t *sQ = smem;
     uint8_t *sK = smem + G::Q_BYTES;
     float *sW = reinterpret_cast<float *>(sK + STAGES * G::K_BYTES);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sW + G::W_FLOATS);
+    int32_t *sTable = reinterpret_cast<int32_t *>(sW + G::W_FLOATS);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sTable + G::TABLE);
     uint64_t *k_full = bars;
     uint64_t *k_empty = bars + STAGES;
     uint64_t *q_full = bars + 2 * STAGES;
@@ -203,7 +205,12 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0 && w_begin < w_end && nblocks > 0) {
+        // The whole warp walks the work list; lane 0 waits on the ring and
+        // issues the copies.  For paged keys the warp stages the batch's
+        // block_table row in shared memory at each block switch, so the
+        // per-tile block lookups are shared-memory reads, not dependent
+        // global loads on the copy path.
+        if (w_begin < w_end && nblocks > 0) {
             Walker w{a.blocks, nblocks, 0, 0, 0, 0, 0};
             w.init(w_begin, w_end);
             int stage = 0, prev_qb = -1;
@@ -211,77 +218,111 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             uint32_t armed = 0, par = 0, q_armed = 0, q_par = 0;
             BlockInfo blk{};
             BatchInfo bi{};
+            bool table_in_smem = false;
+            int ok = 1;
             for (; w.valid(); w.next()) {
                 if (w.qb != prev_qb) {
                     blk = a.blocks[w.qb];
                     bi = a.batches[blk.b];
-                    if (!mbar_wait_bounded(q_empty, qphase ^ 1u, abort_flag, a.timeout_ns)) {
-                        fail(a.hdr, abort_flag, LI_DEV_TIMEOUT);
-                        break;
+                    if (a.is_pa) {
+                        const int need = (bi.Sk + a.block_size - 1) / a.block_size;
+                        table_in_smem = need <= G::TABLE;
+                        __syncwarp();
+                        if (table_in_smem) {
+                            const int32_t *row = a.block_table + (int64_t)blk.b * a.max_blocks_per_seq;
+                            for (int j = lane; j < need; j += 32) sTable[j] = row[j];
+                        }
+                        __syncwarp();
                     }
-                    const int qrow0 = bi.q_off + blk.i0;
-                    if (a.q_box_rows == kQRows) {
-                        mbar_arrive_expect_tx(q_full, CHUNKS * G::Q_CHUNK);
-                        for (int c = 0; c < CHUNKS; ++c)
-                            tma_load_2d(sQ + c * G::Q_CHUNK, &qmap, q_full, c * INNER, qrow0 * a.N1);
-                    } else {
-                        mbar_arrive_expect_tx(q_full, CHUNKS * NQ * a.N1 * kRowBytes);
-                        for (int qi = 0; qi < NQ; ++qi)
-                            for (int c = 0; c < CHUNKS; ++c)
-                                tma_load_2d(sQ + c * G::Q_CHUNK + qi * N1P * kRowBytes, &qmap,
-                                            q_full, c * INNER, (qrow0 + qi) * a.N1);
+                    if (lane == 0) {
+                        if (!mbar_wait_bounded(q_empty, qphase ^ 1u, abort_flag, a.timeout_ns)) {
+                            fail(a.hdr, abort_flag, LI_DEV_TIMEOUT);
+                            ok = 0;
+                        } else {
+                            const int qrow0 = bi.q_off + blk.i0;
+                            if (a.q_box_rows == kQRows) {
+                                mbar_arrive_expect_tx(q_full, CHUNKS * G::Q_CHUNK);
+                                if (a.q_single)
+                                    tma_load_3d(sQ, &qmap, q_full, 0, qrow0 * a.N1, 0);
+                                else
+                                    for (int c = 0; c < CHUNKS; ++c)
+                                        tma_load_2d(sQ + c * G::Q_CHUNK, &qmap, q_full, c * INNER,
+                                                    qrow0 * a.N1);
+                            } else {
+                                mbar_arrive_expect_tx(q_full, CHUNKS * NQ * a.N1 * kRowBytes);
+                                for (int qi = 0; qi < NQ; ++qi)
+                                    for (int c = 0; c < CHUNKS; ++c)
+                                        tma_load_2d(sQ + c * G::Q_CHUNK + qi * N1P * kRowBytes, &qmap,
+                                                    q_full, c * INNER, (qrow0 + qi) * a.N1);
+                            }
+                            q_armed = 1;
+                            q_par = qphase;
+                            qphase ^= 1u;
+                        }
                     }
-                    q_armed = 1;
-                    q_par = qphase;
-                    qphase ^= 1u;
+                    if (!__shfl_sync(0xffffffffu, ok, 0)) break;
                     prev_qb = w.qb;
                 }
-                if (!mbar_wait_bounded(&k_empty[stage], phase ^ 1u, abort_flag, a.timeout_ns)) {
-                    fail(a.hdr, abort_flag, LI_DEV_TIMEOUT);
-                    break;
-                }
-                uint8_t *dst = sK + stage * G::K_BYTES;
-                const int t0 = w.tile * kTileKeys;
-                if (!a.is_pa) {
-                    mbar_arrive_expect_tx(&k_full[stage], G::K_BYTES);
-                    for (int c = 0; c < CHUNKS; ++c)
-                        tma_load_2d(dst + c * G::K_CHUNK, &kmap, &k_full[stage], c * INNER,
-                                    bi.k_off + t0);
-                } else {
-                    // gather the tile from the paged pool, g = pa_box_rows keys at a time
-                    const int g = a.pa_box_rows, nseg = kTileKeys / g;
-                    int blkid[8];
-                    int nvalid = 0;
-                    for (int s = 0; s < nseg; ++s) {
-                        const int t = t0 + s * g;
-                        blkid[s] = -1;
-                        if (t >= bi.Sk) continue;
-                        const int id = a.block_table[(int64_t)blk.b * a.max_blocks_per_seq +
-                                                     t / a.block_size];
-                        if (id < 0 || id >= a.num_blocks) {
-                            atomicOr(&a.hdr->status, LI_DEV_BAD_BLOCK);
-                            continue;
+                if (lane == 0) {
+                    if (!mbar_wait_bounded(&k_empty[stage], phase ^ 1u, abort_flag, a.timeout_ns)) {
+                        fail(a.hdr, abort_flag, LI_DEV_TIMEOUT);
+                        ok = 0;
+                    } else {
+                        uint8_t *dst = sK + stage * G::K_BYTES;
+                        const int t0 = w.tile * kTileKeys;
+                        if (!a.is_pa) {
+                            mbar_arrive_expect_tx(&k_full[stage], G::K_BYTES);
+                            if (a.k_single)
+                                tma_load_3d(dst, &kmap, &k_full[stage], 0, bi.k_off + t0, 0);
+                            else
+                                for (int c = 0; c < CHUNKS; ++c)
+                                    tma_load_2d(dst + c * G::K_CHUNK, &kmap, &k_full[stage],
+                                                c * INNER, bi.k_off + t0);
+                        } else {
+                            // gather the tile from the paged pool, g = pa_box_rows keys at a time
+                            const int g = a.pa_box_rows, nseg = kTileKeys / g;
+                            int blkid[8];
+                            int nvalid = 0;
+                            for (int s = 0; s < nseg; ++s) {
+                                const int t = t0 + s * g;
+                                blkid[s] = -1;
+                                if (t >= bi.Sk) continue;
+                                const int lb = t / a.block_size;
+                                const int id = table_in_smem
+                                                   ? sTable[lb]
+                                                   : a.block_table[(int64_t)blk.b * a.max_blocks_per_seq + lb];
+                                if (id < 0 || id >= a.num_blocks) {
+                                    atomicOr(&a.hdr->status, LI_DEV_BAD_BLOCK);
+                                    continue;
+                                }
+                                blkid[s] = id;
+                                ++nvalid;
+                            }
+                            mbar_arrive_expect_tx(&k_full[stage], nvalid * g * kRowBytes * CHUNKS);
+                            for (int s = 0; s < nseg; ++s) {
+                                if (blkid[s] < 0) continue;
+                                const int t = t0 + s * g;
+                                if (a.k_single)             // g == 128: the whole tile, both chunks
+                                    tma_load_4d(dst, &kmap, &k_full[stage], 0, t % a.block_size, 0,
+                                                blkid[s]);
+                                else
+                                    for (int c = 0; c < CHUNKS; ++c)
+                                        tma_load_3d(dst + c * G::K_CHUNK + s * g * kRowBytes, &kmap,
+                                                    &k_full[stage], c * INNER, t % a.block_size,
+                                                    blkid[s]);
+                            }
                         }
-                        blkid[s] = id;
-                        ++nvalid;
-                    }
-                    mbar_arrive_expect_tx(&k_full[stage], nvalid * g * kRowBytes * CHUNKS);
-                    for (int s = 0; s < nseg; ++s) {
-                        if (blkid[s] < 0) continue;
-                        const int t = t0 + s * g;
-                        for (int c = 0; c < CHUNKS; ++c)
-                            tma_load_3d(dst + c * G::K_CHUNK + s * g * kRowBytes, &kmap,
-                                        &k_full[stage], c * INNER, t % a.block_size, blkid[s]);
+                        armed |= 1u << stage;
+                        par = (par & ~(1u << stage)) | (phase << stage);
+                        if (++stage == STAGES) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
                     }
                 }
-                armed |= 1u << stage;
-                par = (par & ~(1u << stage)) | (phase << stage);
-                if (++stage == STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
+                if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             }
-            if (*abort_flag) {
+            if (lane == 0 && *abort_flag) {
                 // let every copy still in flight land before the CTA exits
                 for (int s = 0; s < STAGES; ++s)
                     if (armed & (1u << s))

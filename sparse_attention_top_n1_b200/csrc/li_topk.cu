@@ -83,6 +83,31 @@ __device__ __forceinline__ T block_exclusive_scan(T v, T *tmp, T &total)
     return r;
 }
 
+__device__ __forceinline__ uint32_t warp_min(uint32_t v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ uint32_t warp_max(uint32_t v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ uint32_t warp_or(uint32_t v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v |= __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ uint32_t warp_and(uint32_t v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v &= __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
 struct RowSrc {
     const float *g;       // row in global memory
     const uint32_t *c;    // row cached as keys in shared memory (or null)
@@ -248,8 +273,12 @@ __device__ void radix_topk(const RowSrc &src, int n, int k, int m, const TopkSme
         __syncthreads();
         uint32_t vor = 0, vand = 0xFFFFFFFFu;
         for (int j = tid; j < m; j += kTopkThreads) { vor |= kin[j]; vand &= kin[j]; }
-        atomicOr(&s_or, vor);
-        atomicAnd(&s_and, vand);
+        vor = warp_or(vor);
+        vand = warp_and(vand);
+        if (lane == 0) {                    // one shared atomic per warp, not per thread
+            atomicOr(&s_or, vor);
+            atomicAnd(&s_and, vand);
+        }
         __syncthreads();
         const uint32_t diff = s_or ^ s_and;
         const int seg = (((m + kWarps - 1) / kWarps) + 31) & ~31;     // elements per warp
@@ -396,7 +425,8 @@ __device__ bool bucket_topk(const RowSrc &src, int n, int k, int m, int kmax, co
         const int d = kBuckets - 1 - (tid * per + e);
         if (d > bstar) lmax = max(lmax, hist[d]);
     }
-    if (lmax) atomicMax(&sh.maxbin, lmax);
+    lmax = warp_max(lmax);
+    if ((tid & 31) == 0 && lmax) atomicMax(&sh.maxbin, lmax);
     __syncthreads();
     if (sh.maxbin > (uint32_t)kBinLimit || cstar > (uint32_t)kCandLimit) return false;
 
@@ -548,8 +578,12 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a)
                 }
         }
     }
-    atomicMin(&sh.kmin, lmin);
-    atomicMax(&sh.kmax, lmax);
+    lmin = warp_min(lmin);
+    lmax = warp_max(lmax);
+    if ((tid & 31) == 0) {                  // one shared atomic per warp, not per thread
+        atomicMin(&sh.kmin, lmin);
+        atomicMax(&sh.kmax, lmax);
+    }
     if (cached) src.c = s.cache;
     __syncthreads();
 

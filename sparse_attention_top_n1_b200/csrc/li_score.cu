@@ -118,6 +118,85 @@ __device__ __forceinline__ float hsum2(uint64_t r)
     return lo + hi;
 }
 
+
+// ReLU, split over two pipes.  max(x, 0) runs on the ALU pipe at half the
+// FP32 rate; x + |x| = 2*ReLU(x) exactly is one FADD on the FMA pipe, with the
+// factor 1/2 folded into that column's weight (a power-of-two scaling, so the
+// product W*ReLU(x) rounds the same).  Three of every eight columns take the
+// FADD form, which balances the two pipes against the packed FMAs.
+constexpr int kFaddPer8 = 3;
+__host__ __device__ constexpr bool fadd_col(int col) { return (col & 7) < kFaddPer8; }
+
+template <int COL>
+__device__ __forceinline__ float relu_c(float x)
+{
+    if constexpr (fadd_col(COL)) return x + fabsf(x);
+    else return fmaxf(x, 0.f);
+}
+
+template <int C, int J, int QPW, int NP2, int N1P>
+__device__ __forceinline__ void epi_group(const float (&v)[32], const uint4 ww, uint64_t (&part)[QPW][NP2])
+{
+    constexpr int q = (C * 32 + J) / N1P;
+    constexpr int p0 = (J / 2) % NP2, p1 = (J / 2 + 1) % NP2;
+    const uint64_t w01 = pack2(__uint_as_float(ww.x), __uint_as_float(ww.y));
+    const uint64_t w23 = pack2(__uint_as_float(ww.z), __uint_as_float(ww.w));
+    part[q][p0] = ffma2(w01, pack2(relu_c<C * 32 + J>(v[J]), relu_c<C * 32 + J + 1>(v[J + 1])), part[q][p0]);
+    part[q][p1] = ffma2(w23, pack2(relu_c<C * 32 + J + 2>(v[J + 2]), relu_c<C * 32 + J + 3>(v[J + 3])), part[q][p1]);
+}
+
+template <int C, int QPW, int NP2, int N1P>
+__device__ __forceinline__ void epi_chunk(const float (&v)[32], const float *myW, uint64_t (&part)[QPW][NP2])
+{
+    const uint4 *w4 = reinterpret_cast<const uint4 *>(myW + C * 32);
+    epi_group<C, 0, QPW, NP2, N1P>(v, w4[0], part);
+    epi_group<C, 4, QPW, NP2, N1P>(v, w4[1], part);
+    epi_group<C, 8, QPW, NP2, N1P>(v, w4[2], part);
+    epi_group<C, 12, QPW, NP2, N1P>(v, w4[3], part);
+    epi_group<C, 16, QPW, NP2, N1P>(v, w4[4], part);
+    epi_group<C, 20, QPW, NP2, N1P>(v, w4[5], part);
+    epi_group<C, 24, QPW, NP2, N1P>(v, w4[6], part);
+    epi_group<C, 28, QPW, NP2, N1P>(v, w4[7], part);
+}
+
+__device__ __forceinline__ void release_acc(uint64_t *bar, int lane)
+{
+    tc_fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar);
+}
+
+// Loads the warp's columns from TMEM two 32-column chunks at a time and
+// reduces them into `part`; hands the accumulator back to the MMA warp once
+// every column is in registers.  NFULL = 4 is the common case of a full query
+// block (no runtime chunk checks); NFULL = 0 takes the chunk count at run time.
+template <int QPW, int NP2, int N1P, int NFULL>
+__device__ __forceinline__ void epi_reduce(uint32_t trow, int nchunks, const float *myW,
+                                           uint64_t (&part)[QPW][NP2], uint64_t *bar, int lane)
+{
+    const int nc = NFULL ? NFULL : nchunks;
+    {
+        float v0[32], v1[32];
+        if (nc > 0) tmem_ld32(trow, v0);
+        if (nc > 1) tmem_ld32(trow + 32, v1);
+        if (nc > 0) {
+            tmem_ld_wait();
+            if (nc <= 2) release_acc(bar, lane);
+        }
+        if (nc > 0) epi_chunk<0, QPW, NP2, N1P>(v0, myW, part);
+        if (nc > 1) epi_chunk<1, QPW, NP2, N1P>(v1, myW, part);
+    }
+    if (nc > 2) {
+        float v0[32], v1[32];
+        tmem_ld32(trow + 64, v0);
+        if (nc > 3) tmem_ld32(trow + 96, v1);
+        tmem_ld_wait();
+        release_acc(bar, lane);
+        epi_chunk<2, QPW, NP2, N1P>(v0, myW, part);
+        if (nc > 3) epi_chunk<3, QPW, NP2, N1P>(v1, myW, part);
+    }
+}
+
 __device__ __forceinline__ float load_weight(const void *w, int dtype, int64_t i)
 {
     if (dtype == LI_FP32) return static_cast<const float *>(w)[i];
@@ -442,7 +521,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                                 wv *= sq;
                             }
                         }
-                        myW[j] = wv;
+                        myW[j] = fadd_col(j) ? 0.5f * wv : wv;
                     }
                     __syncwarp();
                     prev_qb = w.qb;
@@ -476,45 +555,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 for (int q = 0; q < QPW; ++q)
 #pragma unroll
                     for (int p = 0; p < NP2; ++p) part[q][p] = 0ull;
-                // two 32-column chunks per round keep the register footprint
-                // within the 168 registers a 10-warp CTA allows
-#pragma unroll
-                for (int cp = 0; cp < 2; ++cp) {
-                    if (2 * cp < nchunks) {
-                        float v[2][32];
-#pragma unroll
-                        for (int c2 = 0; c2 < 2; ++c2)
-                            if (2 * cp + c2 < nchunks) tmem_ld32(trow + (2 * cp + c2) * 32, v[c2]);
-                        tmem_ld_wait();
-                        if (2 * cp + 2 >= nchunks) {
-                            // every column this warp needs is in registers: hand
-                            // the accumulator back to the MMA warp
-                            tc_fence_before_sync();
-                            __syncwarp();
-                            if (lane == 0) mbar_arrive(&acc_empty[acc]);
-                        }
-#pragma unroll
-                        for (int c2 = 0; c2 < 2; ++c2) {
-                            const int c = 2 * cp + c2;
-                            if (c < nchunks) {
-                                const uint4 *w4 = reinterpret_cast<const uint4 *>(myW + c * 32);
-#pragma unroll
-                                for (int j4 = 0; j4 < 8; ++j4) {
-                                    const uint4 ww = w4[j4];
-                                    const int j = j4 * 4;
-                                    const int q = (c * 32 + j) / N1P;   // same query for j..j+3
-                                    const int p0 = (j / 2) % NP2, p1 = (j / 2 + 1) % NP2;
-                                    const uint64_t w01 = pack2(__uint_as_float(ww.x), __uint_as_float(ww.y));
-                                    const uint64_t w23 = pack2(__uint_as_float(ww.z), __uint_as_float(ww.w));
-                                    part[q][p0] = ffma2(w01, pack2(fmaxf(v[c2][j], 0.f), fmaxf(v[c2][j + 1], 0.f)),
-                                                        part[q][p0]);
-                                    part[q][p1] = ffma2(w23, pack2(fmaxf(v[c2][j + 2], 0.f), fmaxf(v[c2][j + 3], 0.f)),
-                                                        part[q][p1]);
-                                }
-                            }
-                        }
-                    }
-                }
+                if (nchunks == 4 * QPW * N1P / 128)
+                    epi_reduce<QPW, NP2, N1P, 4>(trow, 4, myW, part, &acc_empty[acc], lane);
+                else
+                    epi_reduce<QPW, NP2, N1P, 0>(trow, nchunks, myW, part, &acc_empty[acc], lane);
                 if (nchunks == 0) {                // nothing to read: release at once
                     tc_fence_before_sync();
                     __syncwarp();

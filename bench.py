@@ -6,7 +6,8 @@
 One step is one full indexer call (all three kernels) over one batch of the
 named synthetic workload, with inputs resident in HBM.  The default workload
 is the TileLang test shape (B=2, S1=512, S2=4096, G=32, D=64, k=1024, fp16,
-no mask).  L2 is flushed (a 256 MiB device write) before every timed step,
+no mask).  L2 is flushed before every timed step (a 256 MiB device write,
+then a 256 MiB read of a second buffer so no dirty lines are left behind),
 outside the timed interval; each step is timed with CUDA events on the
 launching stream and the per-step times are summed.  Under torchrun every
 rank runs its own copy of the workload (independent problems, weak scaling,
@@ -326,6 +327,14 @@ def main():
     idx = torch.empty(shape, dtype=torch.int32, device=dev)
     val = torch.empty(shape, dtype=torch.float32, device=dev) if p.return_value else None
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    clean = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def flush_l2():
+        """Evict L2: write a buffer larger than L2, then read a second one, so
+        that the written lines are back in HBM before the next step starts and
+        the timed step does not inherit their write-back."""
+        flush.zero_()
+        clean.sum()
     quant = bool(p.quant)
 
     def call(q, k, w, qs, ks, aq, ak, bt, oi, ov):
@@ -344,7 +353,7 @@ def main():
     t_warm = time.perf_counter()
     nwarm = 0
     while nwarm < args.warmup or (not args.plain and time.perf_counter() - t_warm < 0.8):
-        flush.zero_()
+        flush_l2()
         call(*args_dev)
         nwarm += 1
         if nwarm % 16 == 0:
@@ -372,7 +381,7 @@ def main():
         torch.cuda.synchronize()
         nlaunch = 0
         for s in range(K):
-            flush.zero_()
+            flush_l2()
             if stage_events:
                 li.li_set_profile_events(prof[s])
             starts[s].record()
@@ -442,7 +451,7 @@ def main():
         e_st = [mk() for _ in range(K + args.warmup)]
         e_en = [mk() for _ in range(K + args.warmup)]
         for s in range(K + args.warmup):
-            flush.zero_()
+            flush_l2()
             e_st[s].record()
             for k2, v in host.items():
                 d[k2].copy_(v, non_blocking=True)
@@ -471,7 +480,7 @@ def main():
         "config": {"workload": WORKLOAD_DESC[args.workload], "rows": p.rows,
                    "visible_pairs": counts["pairs"], "sparse_count": p.sparse_count,
                    "return_value": p.return_value,
-                   "l2": "flushed (256 MiB write) before every timed step",
+                   "l2": "flushed before every timed step (256 MiB write, then a 256 MiB read of a second buffer)",
                    "parallelism": "independent replica per GPU" if n > 1 else "1 GPU"},
         "ms_per_step_with_stage_events": (staged_ms / K) if staged_ms else None,
         "effective_tflops": eff_tflops,

@@ -327,7 +327,7 @@ def main():
     idx = torch.empty(shape, dtype=torch.int32, device=dev)
     val = torch.empty(shape, dtype=torch.float32, device=dev) if p.return_value else None
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    clean = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    clean = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)   # fp32: summed without a cast
 
     def flush_l2():
         """Evict L2: write a buffer larger than L2, then read a second one, so

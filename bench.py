@@ -48,11 +48,15 @@ WORKLOAD_DESC = {
     "dsa_prefill": "DSA prefill: B=1 S1=S2=8192 N1=64 D=128 k=2048 mode3 bf16, values on",
     "paged_decode": "paged decode: B=64 S1=1 N1=64 D=128 PA block 128, lengths U[4096,65536], k=2048 mode3 bf16",
     "quant_varlen": "quant varlen TND {2k,4k,8k,16k} N1=64 D=128 fp8 e4m3 + fp32 scales, k=2048 mode3",
+    "quant_varlen_int8": "quant varlen TND {2k,4k,8k,16k} N1=64 D=128 int8 + fp16 scales/weights, k=2048 mode3",
+    "quant_int8_pa": "quant int8 PA (VllmQuant README A3 example): B=24 S1=4 S2=512 N1=64 D=128 block 128, fp16 scales/weights, k=512 mode0",
 }
-RETURN_VALUE = {"tiny": 1, "cfg2": 1, "dsa_prefill": 1, "paged_decode": 0, "quant_varlen": 0}
+RETURN_VALUE = {"tiny": 1, "cfg2": 1, "dsa_prefill": 1, "paged_decode": 0, "quant_varlen": 0,
+                "quant_varlen_int8": 0, "quant_int8_pa": 0}
 
 
-SEEDS = {"tiny": 0, "cfg2": 1, "dsa_prefill": 2, "paged_decode": 3, "quant_varlen": 4}
+SEEDS = {"tiny": 0, "cfg2": 1, "dsa_prefill": 2, "paged_decode": 3, "quant_varlen": 4,
+         "quant_int8_pa": 5, "quant_varlen_int8": 6}
 
 
 def make_workload(name, rank=0):
@@ -102,7 +106,8 @@ def work_counts(p, inp):
     keys_visible = sum(Sk)
     kv_bytes = keys_visible * p.D * es
     compulsory = (nbytes(inp["query"]) + kv_bytes + nbytes(inp["weights"])
-                  + nbytes(inp.get("q_scale")) + keys_visible * 4 * int(p.quant)
+                  + nbytes(inp.get("q_scale"))
+                  + keys_visible * (4 if p.dtype_scale == "fp32" else 2) * int(p.quant)
                   + nbytes(inp.get("block_table")) + nbytes(aq) + nbytes(ak)
                   + p.rows * p.sparse_count * (4 + 4 * p.return_value))
     topk_bytes = rows_nvis * 4 + p.rows * p.sparse_count * (4 + 4 * p.return_value)
@@ -417,7 +422,7 @@ def main():
     score_tflops = counts["flops"] / (avg["score"] * 1e-3) / 1e12
     topk_gbs = counts["topk_bytes"] / (avg["topk"] * 1e-3) / 1e9
     tensor_peak = peaks["bf16_tflops"] * (2.0 if counts["es"] == 1 else 1.0)
-    tensor_note = ("bf16 burst peak x2 (nominal fp8/bf16 ratio), %s" % peak_src
+    tensor_note = ("bf16 burst peak x2 (nominal 8-bit/bf16 ratio, fp8 and int8 alike), %s" % peak_src
                    if counts["es"] == 1 else "bf16 burst peak (fp16 has the same rate), %s" % peak_src)
     kern = {
         "score": {"bound": "tensor", "achieved": score_tflops, "peak": tensor_peak,
@@ -472,7 +477,7 @@ def main():
     if rank == 0 and n == 1 and not (args.no_cpu_baseline or args.plain):
         cpu, _, _ = cpu_oracle_sample(p, inp)
 
-    dtype = {"bf16": "bf16", "fp16": "fp16", "e4m3": "fp8_e4m3"}[p.dtype_qk]
+    dtype = {"bf16": "bf16", "fp16": "fp16", "e4m3": "fp8_e4m3", "int8": "int8"}[p.dtype_qk]
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": n, "steps": K,
         "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,

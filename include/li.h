@@ -71,9 +71,9 @@ typedef enum { LI_BSND = 0, LI_TND = 1, LI_PA_BSND = 2 } li_layout;
  *   layout_k       LI_BSND: key [B,S2,N2,D]; LI_TND: key [T2,N2,D];
  *                  LI_PA_BSND: key [num_blocks,block_size,N2,D] addressed via block_table.
  *                  Without PA, layout_k must equal layout_q.
- *   dtype_qk       LI_BF16 / LI_FP16 (li_indexer), LI_FP8_E4M3 (li_quant_indexer)
+ *   dtype_qk       LI_BF16 / LI_FP16 (li_indexer); LI_FP8_E4M3 / LI_INT8 (li_quant_indexer)
  *   dtype_w        LI_BF16 / LI_FP16 / LI_FP32
- *   dtype_scale    LI_FP32 (li_quant_indexer only)
+ *   dtype_scale    LI_FP32 / LI_FP16 (li_quant_indexer only)
  *   N1             query heads, 1..64;  N2 key heads, must be 1
  *   D              head dim: 128, or 64 for 16-bit q/k (the TileLang test shape)
  *   num_blocks, block_size, max_blocks_per_seq
@@ -134,17 +134,18 @@ LI_API li_status li_indexer(const li_params *p, const void *query, const void *k
                      void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * The quantised indexer (VllmQuantLightningIndexer README, "功能说明"):
- * q/k are fp8 e4m3, and the per-token-head dequant scales multiply the dot
- * product before the ReLU.
- *   q_scale  fp32, same layout as weights ([B,S1,N1] or [T1,N1])
- *   k_scale  fp32 per key token: [B,S2,N2], [T2,N2] or [num_blocks,block_size,N2]
+ * The quantised indexer (VllmQuantLightningIndexer README, "功能说明" and
+ * "参数说明"): q/k are fp8 e4m3 or int8, and the per-token-head dequant
+ * scales multiply the dot product before the ReLU.  int8 q/k accumulate
+ * exactly in s32 (|q.k| <= 2^21 for D = 128) and are converted to fp32.
+ *   q_scale  dtype_scale (fp32 or fp16), same layout as weights ([B,S1,N1] or [T1,N1])
+ *   k_scale  dtype_scale per key token: [B,S2,N2], [T2,N2] or [num_blocks,block_size,N2]
  * Scales must be >= 0 (then ReLU(sq*sk*x) = sq*sk*ReLU(x), which the kernel
  * uses); a negative scale is flagged with LI_DEV_NEG_SCALE.  Other arguments
  * as li_indexer.
  */
 LI_API li_status li_quant_indexer(const li_params *p, const void *query, const void *key,
-                           const void *weights, const float *q_scale, const float *k_scale,
+                           const void *weights, const void *q_scale, const void *k_scale,
                            const int32_t *act_seq_q, const int32_t *act_seq_k,
                            const int32_t *block_table, int32_t *sparse_indices,
                            float *sparse_values, void *workspace, size_t workspace_bytes,

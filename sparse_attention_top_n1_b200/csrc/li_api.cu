@@ -90,14 +90,11 @@ li_status check_params(const li_params *pp, bool quant)
         return fail(LI_ERR_SHAPE, "return_value must be 0 or 1");
     if (p.max_seqlen_k < 0) return fail(LI_ERR_SHAPE, "max_seqlen_k must be >= 0");
     if (quant) {
-        if (p.dtype_qk == LI_INT8)
-            return fail(LI_ERR_UNSUPPORTED, "int8 query/key is not built yet (fp8 e4m3 only)");
-        if (p.dtype_qk != LI_FP8_E4M3)
-            return fail(LI_ERR_DTYPE, "li_quant_indexer takes fp8 e4m3 query/key");
-        if (p.dtype_scale == LI_FP16)
-            return fail(LI_ERR_UNSUPPORTED, "fp16 dequant scales are not built yet");
-        if (p.dtype_scale != LI_FP32) return fail(LI_ERR_DTYPE, "dequant scales must be fp32");
-        if (p.D != 128) return fail(LI_ERR_SHAPE, "D must be 128 for fp8 query/key");
+        if (p.dtype_qk != LI_FP8_E4M3 && p.dtype_qk != LI_INT8)
+            return fail(LI_ERR_DTYPE, "li_quant_indexer takes fp8 e4m3 or int8 query/key");
+        if (p.dtype_scale != LI_FP32 && p.dtype_scale != LI_FP16)
+            return fail(LI_ERR_DTYPE, "dequant scales must be fp32 or fp16");
+        if (p.D != 128) return fail(LI_ERR_SHAPE, "D must be 128 for 8-bit query/key");
     } else {
         if (p.dtype_qk != LI_BF16 && p.dtype_qk != LI_FP16)
             return fail(LI_ERR_DTYPE, "li_indexer takes bf16 or fp16 query/key");
@@ -220,7 +217,7 @@ int topk_cap(int64_t ld, int k, int kmax)
 }
 
 li_status run(const li_params *pp, bool quant, const void *query, const void *key,
-              const void *weights, const float *q_scale, const float *k_scale,
+              const void *weights, const void *q_scale, const void *k_scale,
               const int32_t *act_q, const int32_t *act_k, const int32_t *block_table,
               int32_t *out_idx, float *out_val, void *workspace, size_t ws_bytes, void *stream)
 {
@@ -243,6 +240,9 @@ li_status run(const li_params *pp, bool quant, const void *query, const void *ke
         return fail(LI_ERR_SHAPE, "query and key must be 16-byte aligned");
     if (!aligned(weights, 4) || !aligned(out_idx, 4) || (out_val && !aligned(out_val, 4)))
         return fail(LI_ERR_SHAPE, "weights and outputs must be 4-byte aligned");
+    if (quant && (!aligned(q_scale, p.dtype_scale == LI_FP32 ? 4 : 2) ||
+                  !aligned(k_scale, p.dtype_scale == LI_FP32 ? 4 : 2)))
+        return fail(LI_ERR_SHAPE, "dequant scales must be aligned to their element size");
     const Tiling t = make_tiling(p);
     const WorkspaceLayout w = make_layout(p, t);
     if (!workspace) return fail(LI_ERR_WORKSPACE, "workspace is NULL");
@@ -362,10 +362,14 @@ li_status run(const li_params *pp, bool quant, const void *query, const void *ke
     sa.q_box_rows = q_box_rows;
     sa.q_single = q_single;
     sa.k_single = k_single;
-    const uint32_t fmt = quant ? 0u : (p.dtype_qk == LI_BF16 ? 1u : 0u);
-    sa.idesc_base = make_idesc(fmt, fmt, 128, 0);
+    // operand formats: f16 0 / bf16 1 (kind::f16), e4m3 0 (kind::f8f6f4),
+    // signed 8-bit 1 with an s32 accumulator (kind::i8)
+    const int kind = !quant ? kKindF16 : (p.dtype_qk == LI_INT8 ? kKindI8 : kKindE4M3);
+    const uint32_t fmt = kind == kKindF16 ? (p.dtype_qk == LI_BF16 ? 1u : 0u) : (kind == kKindI8 ? 1u : 0u);
+    sa.idesc_base = make_idesc(fmt, fmt, 128, 0, kind == kKindI8 ? 2u : 1u);
+    sa.dtype_scale = p.dtype_scale;
     sa.timeout_ns = kDefaultTimeoutNs;
-    e = launch_score(sa, t, qmap, kmap, quant ? 1 : 0, sms, s);
+    e = launch_score(sa, t, qmap, kmap, kind, sms, s);
     if (e != cudaSuccess) return fail(LI_ERR_CUDA, "score launch: %s", cudaGetErrorString(e));
     ++g_launches;
     if (!prof_mark(2, s)) return fail(LI_ERR_CUDA, "recording profile event 2 failed");
@@ -406,7 +410,7 @@ extern "C" {
 li_status li_output_shape(const li_params *p, int64_t out_dims[4], int32_t *ndim)
 {
     if (!out_dims || !ndim) return fail(LI_ERR_NULL, "out_dims and ndim are required");
-    li_status st = check_params(p, p && p->dtype_qk == LI_FP8_E4M3);
+    li_status st = check_params(p, p && (p->dtype_qk == LI_FP8_E4M3 || p->dtype_qk == LI_INT8));
     if (st != LI_OK) return st;
     if (p->layout_q == LI_BSND) {
         out_dims[0] = p->B;
@@ -427,7 +431,7 @@ li_status li_output_shape(const li_params *p, int64_t out_dims[4], int32_t *ndim
 li_status li_workspace_size(const li_params *p, size_t *bytes)
 {
     if (!bytes) return fail(LI_ERR_NULL, "bytes is NULL");
-    li_status st = check_params(p, p && p->dtype_qk == LI_FP8_E4M3);
+    li_status st = check_params(p, p && (p->dtype_qk == LI_FP8_E4M3 || p->dtype_qk == LI_INT8));
     if (st != LI_OK) return st;
     *bytes = make_layout(*p, make_tiling(*p)).total;
     return LI_OK;
@@ -443,7 +447,7 @@ li_status li_indexer(const li_params *p, const void *query, const void *key, con
 }
 
 li_status li_quant_indexer(const li_params *p, const void *query, const void *key,
-                           const void *weights, const float *q_scale, const float *k_scale,
+                           const void *weights, const void *q_scale, const void *k_scale,
                            const int32_t *act_seq_q, const int32_t *act_seq_k,
                            const int32_t *block_table, int32_t *sparse_indices,
                            float *sparse_values, void *workspace, size_t workspace_bytes,

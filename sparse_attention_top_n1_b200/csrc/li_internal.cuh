@@ -81,8 +81,8 @@ struct PlanArgs {
 
 struct ScoreArgs {
     const void *weights;
-    const float *q_scale;
-    const float *k_scale;
+    const void *q_scale;        // dequant scales, dtype_scale (fp32 or fp16)
+    const void *k_scale;
     const int32_t *block_table;
     const BatchInfo *batches;
     const BlockInfo *blocks;
@@ -90,7 +90,7 @@ struct ScoreArgs {
     float *scores;
     int64_t ld;
     int32_t N1, mode, is_pa, quant;
-    int32_t dtype_w;
+    int32_t dtype_w, dtype_scale;
     int32_t block_size, max_blocks_per_seq, num_blocks, pa_box_rows;
     int32_t q_box_rows;         // rows per Q TMA box: n1p*nq (packed) or N1 (per query)
     int32_t q_single, k_single; // one copy covers both 128-byte chunks (3-D / 4-D maps)
@@ -117,8 +117,10 @@ size_t score_smem_bytes(int chunks);
 int score_stages(int chunks);
 
 cudaError_t launch_plan(const PlanArgs &a, cudaStream_t s);
+// Operand kinds of the score MMA.
+enum ScoreKind { kKindF16 = 0, kKindE4M3 = 1, kKindI8 = 2 };
 cudaError_t launch_score(const ScoreArgs &a, const Tiling &t, const CUtensorMap &qmap,
-                         const CUtensorMap &kmap, int fp8, int grid, cudaStream_t s);
+                         const CUtensorMap &kmap, int kind, int grid, cudaStream_t s);
 cudaError_t launch_topk(const TopkArgs &a, cudaStream_t s);
 cudaError_t launch_wait_selftest(int32_t *status, int64_t timeout_ns, cudaStream_t s);
 

@@ -104,11 +104,38 @@ __device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c)
     return d;
 }
 
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 __device__ __forceinline__ uint64_t pack2(float lo, float hi)
 {
     uint64_t r;
     asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
     return r;
+}
+
+__device__ __forceinline__ void unpack2(uint64_t r, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+
+// s32 accumulator bits (as loaded from TMEM) to fp32, in place.  Exact for
+// |x| < 2^22 (an int8 dot product over D = 128 is at most 2^21): the bit
+// pattern of 1.5*2^23 plus x is the float 1.5*2^23 + x, and subtracting
+// 1.5*2^23 leaves x.
+__device__ __forceinline__ void s32_to_f32(float (&v)[32])
+{
+    const uint64_t m2 = pack2(-12582912.f, -12582912.f);
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+        const float a = __int_as_float(__float_as_int(v[i]) + 0x4B400000);
+        const float b = __int_as_float(__float_as_int(v[i + 1]) + 0x4B400000);
+        unpack2(fadd2(pack2(a, b), m2), v[i], v[i + 1]);
+    }
 }
 
 __device__ __forceinline__ float hsum2(uint64_t r)
@@ -170,10 +197,11 @@ __device__ __forceinline__ void release_acc(uint64_t *bar, int lane)
 // reduces them into `part`; hands the accumulator back to the MMA warp once
 // every column is in registers.  NFULL = 4 is the common case of a full query
 // block (no runtime chunk checks); NFULL = 0 takes the chunk count at run time.
-template <int QPW, int NP2, int N1P, int NFULL>
+template <int QPW, int NP2, int N1P, int NFULL, int KIND>
 __device__ __forceinline__ void epi_reduce(uint32_t trow, int nchunks, const float *myW,
                                            uint64_t (&part)[QPW][NP2], uint64_t *bar, int lane)
 {
+    constexpr bool S32 = KIND == kKindI8;       // integer accumulator
     const int nc = NFULL ? NFULL : nchunks;
     {
         float v0[32], v1[32];
@@ -182,6 +210,10 @@ __device__ __forceinline__ void epi_reduce(uint32_t trow, int nchunks, const flo
         if (nc > 0) {
             tmem_ld_wait();
             if (nc <= 2) release_acc(bar, lane);
+            if constexpr (S32) {
+                s32_to_f32(v0);
+                if (nc > 1) s32_to_f32(v1);
+            }
         }
         if (nc > 0) epi_chunk<0, QPW, NP2, N1P>(v0, myW, part);
         if (nc > 1) epi_chunk<1, QPW, NP2, N1P>(v1, myW, part);
@@ -192,6 +224,10 @@ __device__ __forceinline__ void epi_reduce(uint32_t trow, int nchunks, const flo
         if (nc > 3) tmem_ld32(trow + 96, v1);
         tmem_ld_wait();
         release_acc(bar, lane);
+        if constexpr (S32) {
+            s32_to_f32(v0);
+            if (nc > 3) s32_to_f32(v1);
+        }
         epi_chunk<2, QPW, NP2, N1P>(v0, myW, part);
         if (nc > 3) epi_chunk<3, QPW, NP2, N1P>(v1, myW, part);
     }
@@ -205,13 +241,19 @@ __device__ __forceinline__ float load_weight(const void *w, int dtype, int64_t i
     return __half2float(__ushort_as_half(h));
 }
 
+__device__ __forceinline__ float load_scale(const void *p, int dtype, int64_t i)
+{
+    if (dtype == LI_FP32) return static_cast<const float *>(p)[i];
+    return __half2float(__ushort_as_half(static_cast<const unsigned short *>(p)[i]));
+}
+
 __device__ __forceinline__ void fail(PlanHeader *hdr, volatile int *abort_flag, int bit)
 {
     atomicOr(&hdr->status, bit);
     *abort_flag = 1;
 }
 
-template <int CHUNKS, int N1P, bool FP8>
+template <int CHUNKS, int N1P, int KIND>
 __global__ void __launch_bounds__(kScoreThreads, 1)
     score_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                  const ScoreArgs a)
@@ -221,7 +263,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     constexpr int NQ = 256 / N1P;                 // queries per block
     constexpr int QPW = 128 / N1P;                // queries per epilogue warp half
     constexpr int NP2 = N1P >= 32 ? 4 : (N1P == 16 ? 2 : 1);  // packed partial sums per query
-    constexpr int INNER = FP8 ? 128 : 64;         // elements per 128-byte row chunk
+    constexpr int INNER = KIND == kKindF16 ? 64 : 128;   // elements per 128-byte row chunk
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -448,8 +490,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint64_t ad = smem_desc_sw128(k_addr + c * G::K_CHUNK + kk * 32);
                         const uint64_t bd = smem_desc_sw128(sQ_addr + c * G::Q_CHUNK + kk * 32);
-                        if (FP8)
+                        if constexpr (KIND == kKindE4M3)
                             mma_f8(d_tmem, ad, bd, idesc, (c | kk) != 0);
+                        else if constexpr (KIND == kKindI8)
+                            mma_i8(d_tmem, ad, bd, idesc, (c | kk) != 0);
                         else
                             mma_f16(d_tmem, ad, bd, idesc, (c | kk) != 0);
                     }
@@ -516,7 +560,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                             const int64_t r = (int64_t)(bi.q_off + i) * a.N1 + h;
                             wv = load_weight(a.weights, a.dtype_w, r);
                             if (a.quant) {
-                                const float sq = a.q_scale[r];
+                                const float sq = load_scale(a.q_scale, a.dtype_scale, r);
                                 if (sq < 0.f) atomicOr(&a.hdr->status, LI_DEV_NEG_SCALE);
                                 wv *= sq;
                             }
@@ -546,7 +590,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                             kr = (int64_t)id * a.block_size + t % a.block_size;
                     }
                     if (kr >= 0) {
-                        ks = a.k_scale[kr];
+                        ks = load_scale(a.k_scale, a.dtype_scale, kr);
                         if (ks < 0.f) atomicOr(&a.hdr->status, LI_DEV_NEG_SCALE);
                     }
                 }
@@ -556,9 +600,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 #pragma unroll
                     for (int p = 0; p < NP2; ++p) part[q][p] = 0ull;
                 if (nchunks == 4 * QPW * N1P / 128)
-                    epi_reduce<QPW, NP2, N1P, 4>(trow, 4, myW, part, &acc_empty[acc], lane);
+                    epi_reduce<QPW, NP2, N1P, 4, KIND>(trow, 4, myW, part, &acc_empty[acc], lane);
                 else
-                    epi_reduce<QPW, NP2, N1P, 0>(trow, nchunks, myW, part, &acc_empty[acc], lane);
+                    epi_reduce<QPW, NP2, N1P, 0, KIND>(trow, nchunks, myW, part, &acc_empty[acc], lane);
                 if (nchunks == 0) {                // nothing to read: release at once
                     tc_fence_before_sync();
                     __syncwarp();
@@ -592,11 +636,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     if (warp == 1) tmem_dealloc(tmem_base, 2 * kAccCols);
 }
 
-template <int CHUNKS, int N1P, bool FP8>
+template <int CHUNKS, int N1P, int KIND>
 cudaError_t launch_one(const ScoreArgs &a, const CUtensorMap &qmap, const CUtensorMap &kmap,
                        int grid, cudaStream_t s)
 {
-    auto kern = score_kernel<CHUNKS, N1P, FP8>;
+    auto kern = score_kernel<CHUNKS, N1P, KIND>;
     const size_t smem = Geometry<CHUNKS>::SMEM;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -613,15 +657,15 @@ cudaError_t launch_one(const ScoreArgs &a, const CUtensorMap &qmap, const CUtens
     return cudaLaunchKernelEx(&cfg, kern, qmap, kmap, a);
 }
 
-template <int CHUNKS, bool FP8>
+template <int CHUNKS, int KIND>
 cudaError_t launch_n1p(const ScoreArgs &a, int n1p, const CUtensorMap &qmap,
                        const CUtensorMap &kmap, int grid, cudaStream_t s)
 {
     switch (n1p) {
-    case 8: return launch_one<CHUNKS, 8, FP8>(a, qmap, kmap, grid, s);
-    case 16: return launch_one<CHUNKS, 16, FP8>(a, qmap, kmap, grid, s);
-    case 32: return launch_one<CHUNKS, 32, FP8>(a, qmap, kmap, grid, s);
-    case 64: return launch_one<CHUNKS, 64, FP8>(a, qmap, kmap, grid, s);
+    case 8: return launch_one<CHUNKS, 8, KIND>(a, qmap, kmap, grid, s);
+    case 16: return launch_one<CHUNKS, 16, KIND>(a, qmap, kmap, grid, s);
+    case 32: return launch_one<CHUNKS, 32, KIND>(a, qmap, kmap, grid, s);
+    case 64: return launch_one<CHUNKS, 64, KIND>(a, qmap, kmap, grid, s);
     }
     return cudaErrorInvalidValue;
 }
@@ -632,12 +676,14 @@ size_t score_smem_bytes(int chunks) { return chunks == 2 ? Geometry<2>::SMEM : G
 int score_stages(int chunks) { return chunks == 2 ? Geometry<2>::STAGES : Geometry<1>::STAGES; }
 
 cudaError_t launch_score(const ScoreArgs &a, const Tiling &t, const CUtensorMap &qmap,
-                         const CUtensorMap &kmap, int fp8, int grid, cudaStream_t s)
+                         const CUtensorMap &kmap, int kind, int grid, cudaStream_t s)
 {
-    if (fp8) return t.chunks == 1 ? launch_n1p<1, true>(a, t.n1p, qmap, kmap, grid, s)
-                                  : cudaErrorInvalidValue;
-    return t.chunks == 2 ? launch_n1p<2, false>(a, t.n1p, qmap, kmap, grid, s)
-                         : launch_n1p<1, false>(a, t.n1p, qmap, kmap, grid, s);
+    if (kind == kKindE4M3)
+        return t.chunks == 1 ? launch_n1p<1, kKindE4M3>(a, t.n1p, qmap, kmap, grid, s) : cudaErrorInvalidValue;
+    if (kind == kKindI8)
+        return t.chunks == 1 ? launch_n1p<1, kKindI8>(a, t.n1p, qmap, kmap, grid, s) : cudaErrorInvalidValue;
+    return t.chunks == 2 ? launch_n1p<2, kKindF16>(a, t.n1p, qmap, kmap, grid, s)
+                         : launch_n1p<1, kKindF16>(a, t.n1p, qmap, kmap, grid, s);
 }
 
 }  // namespace li

@@ -208,6 +208,18 @@ __device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_
         : "memory");
 }
 
+// D[tmem] (+)= A * B^T on signed 8-bit operands with an s32 accumulator.
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 operation issued so far by this
 // thread has completed.
 __device__ __forceinline__ void mma_commit(uint64_t *bar)
@@ -263,9 +275,9 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr)
 // Instruction descriptor: dense, fp32 accumulator, A/B K-major.
 //   a_fmt/b_fmt: kind::f16 -> 0 = f16, 1 = bf16; kind::f8f6f4 -> 0 = e4m3.
 __host__ __device__ constexpr uint32_t make_idesc(uint32_t a_fmt, uint32_t b_fmt, uint32_t M,
-                                                  uint32_t N)
+                                                  uint32_t N, uint32_t d_fmt = 1u)
 {
-    return (1u << 4)                 // D format: f32
+    return (d_fmt << 4)              // D format: 1 = f32, 2 = s32
            | (a_fmt << 7) | (b_fmt << 10)
            | ((N >> 3) << 17)       // N / 8
            | ((M >> 4) << 24);      // M / 16

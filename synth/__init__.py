@@ -21,6 +21,12 @@ named by the pages:
 * ``quant_varlen`` -- TND fp8-e4m3 q/k with per-token-head absmax scales
                       (VllmQuantLightningIndexer README, "功能说明"), 4
                       sequences of 2048/4096/8192/16384 tokens.
+* ``quant_varlen_int8`` -- the same sequences with int8 q/k and fp16 scales
+                      and weights (the README's A2/A3 dtypes, "参数说明").
+* ``quant_int8_pa`` -- the README's A3 call example ("Atlas A3 推理系列产品调用
+                      说明"): B=24, S1=4, S2=512, PA_BSND block 128, int8 q/k
+                      uniform over the int8 range, fp16 scales U[0, 10], fp16
+                      weights U[0, 0.01], k=512, mask 0.
 """
 from __future__ import annotations
 
@@ -37,6 +43,7 @@ DTYPES = {
     "int8": torch.int8,
 }
 E4M3_MAX = 448.0
+INT8_MAX = 127.0
 INT64_MAX = (1 << 63) - 1
 
 
@@ -100,6 +107,22 @@ def quantize_e4m3_per_row(x: torch.Tensor):
 # --------------------------------------------------------------------------
 # The named workloads
 # --------------------------------------------------------------------------
+
+def quantize_int8_per_row(x: torch.Tensor):
+    """Per-(token, head) absmax quantisation to int8 (input recipe).
+
+    scale = absmax(x[..., :]) / 127 (1 where the absmax is 0); the stored code
+    is round-half-to-even of x / scale, clamped to [-127, 127].  Returns
+    (codes, scale) with fp32 scales.
+    """
+    amax = x.abs().amax(dim=-1)
+    scale = torch.where(amax > 0, amax / INT8_MAX, torch.ones_like(amax))
+    codes = torch.round(x / scale.unsqueeze(-1)).clamp(-INT8_MAX, INT8_MAX).to(torch.int8)
+    return codes, scale.to(torch.float32)
+
+
+QUANTIZERS = {"e4m3": quantize_e4m3_per_row, "int8": quantize_int8_per_row}
+
 
 def make_tiny(seed: int = 0):
     p = Problem(layout_q="BSND", layout_k="BSND", dtype_qk="bf16", dtype_w="bf16",
@@ -170,23 +193,59 @@ def make_paged_decode(seed: int = 3, B: int = 64, lo: int = 4096, hi: int = 6553
 
 
 def make_quant_varlen(seed: int = 4, lens=(2048, 4096, 8192, 16384), return_value: int = 0,
-                      sparse_count: int = 2048):
-    """TND fp8 e4m3 q/k with fp32 per-token-head dequant scales, fp32 weights."""
+                      sparse_count: int = 2048, qdtype: str = "e4m3", dtype_scale: str = "fp32",
+                      dtype_w: str = "fp32"):
+    """TND 8-bit q/k (fp8 e4m3 or int8) with per-token-head dequant scales."""
     N1, D = 64, 128
     T = int(sum(lens))
     g = _gen(seed)
     xq = torch.randn(T, N1, D, generator=g, dtype=torch.float32)
     xk = torch.randn(T, 1, D, generator=g, dtype=torch.float32)
-    w = torch.randn(T, N1, generator=g, dtype=torch.float32)
-    q, qs = quantize_e4m3_per_row(xq)
-    k, ks = quantize_e4m3_per_row(xk)
+    w = torch.randn(T, N1, generator=g, dtype=torch.float32).to(DTYPES[dtype_w])
+    q, qs = QUANTIZERS[qdtype](xq)
+    k, ks = QUANTIZERS[qdtype](xk)
+    qs, ks = qs.to(DTYPES[dtype_scale]), ks.to(DTYPES[dtype_scale])
     cum = torch.tensor(lens, dtype=torch.int64).cumsum(0).to(torch.int32)
-    p = Problem(layout_q="TND", layout_k="TND", dtype_qk="e4m3", dtype_w="fp32",
-                dtype_scale="fp32", quant=True, B=len(lens), T1=T, T2=T, N1=N1, N2=1,
+    p = Problem(layout_q="TND", layout_k="TND", dtype_qk=qdtype, dtype_w=dtype_w,
+                dtype_scale=dtype_scale, quant=True, B=len(lens), T1=T, T2=T, N1=N1, N2=1,
                 D=D, sparse_count=sparse_count, sparse_mode=3, return_value=return_value,
                 max_seqlen_k=int(max(lens)))
     return p, dict(query=q, key=k, weights=w, q_scale=qs, k_scale=ks,
                    act_q=cum.clone(), act_k=cum.clone())
+
+
+def make_quant_varlen_int8(seed: int = 6, return_value: int = 0):
+    """quant_varlen with int8 q/k, fp16 scales and fp16 weights."""
+    return make_quant_varlen(seed=seed, return_value=return_value, qdtype="int8",
+                             dtype_scale="fp16", dtype_w="fp16")
+
+
+def make_quant_int8_pa(seed: int = 5, B: int = 24, S1: int = 4, S2: int = 512,
+                       block_size: int = 128, sparse_count: int = 512, sparse_mode: int = 0,
+                       return_value: int = 1):
+    """The README's A3 example call: int8 q/k over the int8 range, fp16 scales
+    in [0, 10), fp16 weights in [0, 0.01), PA_BSND keys whose block table maps
+    logical block j of batch b to physical block b*max_blocks + j.
+
+    Draw order: key, key scales, query, query scales, weights.
+    """
+    N1, D = 64, 128
+    g = _gen(seed)
+    mb = (S2 + block_size - 1) // block_size
+    table = torch.arange(B * mb, dtype=torch.int32).reshape(B, mb)
+    key = torch.randint(-128, 128, (B * mb, block_size, 1, D), generator=g, dtype=torch.int64).to(torch.int8)
+    ks = (torch.rand(B * mb, block_size, 1, generator=g) * 10).to(torch.float16)
+    q = torch.randint(-128, 128, (B, S1, N1, D), generator=g, dtype=torch.int64).to(torch.int8)
+    qs = (torch.rand(B, S1, N1, generator=g) * 10).to(torch.float16)
+    w = (torch.rand(B, S1, N1, generator=g) * 0.01).to(torch.float16)
+    p = Problem(layout_q="BSND", layout_k="PA_BSND", dtype_qk="int8", dtype_w="fp16",
+                dtype_scale="fp16", quant=True, B=B, S1=S1, S2=0, N1=N1, N2=1, D=D,
+                num_blocks=B * mb, block_size=block_size, max_blocks_per_seq=mb,
+                sparse_count=sparse_count, sparse_mode=sparse_mode, return_value=return_value,
+                max_seqlen_k=S2)
+    lens = torch.full((B,), S2, dtype=torch.int32)
+    return p, dict(query=q, key=key, weights=w, q_scale=qs, k_scale=ks, act_q=torch.full((B,), S1, dtype=torch.int32),
+                   act_k=lens, block_table=table)
 
 
 WORKLOADS = {
@@ -195,6 +254,8 @@ WORKLOADS = {
     "dsa_prefill": make_dsa_prefill,
     "paged_decode": make_paged_decode,
     "quant_varlen": make_quant_varlen,
+    "quant_varlen_int8": make_quant_varlen_int8,
+    "quant_int8_pa": make_quant_int8_pa,
 }
 
 
@@ -205,7 +266,8 @@ WORKLOADS = {
 def make_random(seed: int, *, layout_q="BSND", layout_k="BSND", dtype_qk="bf16",
                 dtype_w="bf16", B=2, S1=40, S2=300, N1=8, D=128, sparse_count=64,
                 sparse_mode=3, return_value=1, ragged=True, block_size=64,
-                quant=False, empty_rows=False, key_block_pad=0):
+                quant=False, empty_rows=False, key_block_pad=0, quant_dtype="e4m3",
+                dtype_scale="fp32"):
     """A random problem of the given layout; lengths are ragged when asked.
 
     BSND: actual lengths in [1, S] (or S when not ragged).  TND: per-sequence
@@ -282,14 +344,14 @@ def make_random(seed: int, *, layout_q="BSND", layout_k="BSND", dtype_qk="bf16",
         if key_block_pad:
             p.key_block_stride = (block_size + key_block_pad) * N2 * D
     if quant:
-        q, qs = quantize_e4m3_per_row(xq)
-        k, ks = quantize_e4m3_per_row(xk)
-        inputs["q_scale"] = qs
+        q, qs = QUANTIZERS[quant_dtype](xq)
+        k, ks = QUANTIZERS[quant_dtype](xk)
+        inputs["q_scale"] = qs.to(DTYPES[dtype_scale])
         if layout_k == "PA_BSND":
             ks = ks[:, :block_size].contiguous()      # [blocks, block_size, N2]
-        inputs["k_scale"] = ks
-        p.dtype_qk = "e4m3"
-        p.dtype_scale = "fp32"
+        inputs["k_scale"] = ks.to(DTYPES[dtype_scale])
+        p.dtype_qk = quant_dtype
+        p.dtype_scale = dtype_scale
     else:
         q = xq.to(DTYPES[qdt])
         k = xk.to(DTYPES[qdt])

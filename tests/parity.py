@@ -1,6 +1,6 @@
 """Element-by-element comparison of the CUDA path with the fp64 oracle.
 
-The rule (tolerance |g - o| <= atol + rtol*|o|; bf16/fp16: rtol 2e-3, atol
+The rule (tolerance |g - o| <= atol + rtol*|o|; bf16/fp16/int8: rtol 2e-3, atol
 1e-4; fp8: rtol 5e-2, atol 1e-4):
   * slots past min(k, visible) hold index -1 and value -inf, bit for bit;
   * the valid indices are distinct and visible (0 <= t < nvis);
@@ -18,7 +18,7 @@ import torch
 
 import oracle
 
-TOL = {"bf16": (2e-3, 1e-4), "fp16": (2e-3, 1e-4), "e4m3": (5e-2, 1e-4)}
+TOL = {"bf16": (2e-3, 1e-4), "fp16": (2e-3, 1e-4), "e4m3": (5e-2, 1e-4), "int8": (2e-3, 1e-4)}
 NEG_INF_BITS = np.float32(-np.inf).view(np.uint32)
 
 

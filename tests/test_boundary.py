@@ -111,10 +111,14 @@ def test_quant_checks():
     st = L.li_quant_indexer(ctypes.byref(pr), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None,
                             FAKE, None, FAKE, 1 << 40, None)
     assert li.STATUS_NAMES[st] == "LI_ERR_DTYPE"
-    pr = _base(dtype_qk="int8")
+    pr = _base(dtype_qk="int8", D=64)
     st = L.li_quant_indexer(ctypes.byref(pr), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None,
                             FAKE, None, FAKE, 1 << 40, None)
-    assert li.STATUS_NAMES[st] == "LI_ERR_UNSUPPORTED"
+    assert li.STATUS_NAMES[st] == "LI_ERR_SHAPE"
+    pr = _base(dtype_qk="int8", dtype_scale="bf16")
+    st = L.li_quant_indexer(ctypes.byref(pr), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None,
+                            FAKE, None, FAKE, 1 << 40, None)
+    assert li.STATUS_NAMES[st] == "LI_ERR_DTYPE"
     pr = _base(dtype_qk="e4m3", D=64)
     st = L.li_quant_indexer(ctypes.byref(pr), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None,
                             FAKE, None, FAKE, 1 << 40, None)

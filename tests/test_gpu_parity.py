@@ -74,6 +74,12 @@ CASES = {
     "quant_pa": dict(layout_k="PA_BSND", quant=True, dtype_w="fp32", block_size=64, N1=64,
                      sparse_mode=3),
     "quant_bsnd_n8": dict(quant=True, dtype_w="fp32", sparse_mode=0),
+    "int8_tnd_fp16": dict(layout_q="TND", layout_k="TND", quant=True, quant_dtype="int8",
+                          dtype_scale="fp16", dtype_w="fp16", N1=64, S1=60, S2=300, sparse_mode=3),
+    "int8_pa_fp32": dict(layout_k="PA_BSND", quant=True, quant_dtype="int8", dtype_w="fp32",
+                         block_size=32, N1=64, sparse_mode=3),
+    "int8_bsnd_n5": dict(quant=True, quant_dtype="int8", dtype_scale="fp16", dtype_w="bf16",
+                         N1=5, sparse_mode=0),
 }
 
 
@@ -86,7 +92,8 @@ def test_small_case_parity(name):
 
 
 @pytest.mark.parametrize("name", ["bsnd_mode3", "bsnd_fp16_d64_n32", "tnd_mode3", "pa48",
-                                  "bsnd_n3_padded_heads", "quant_tnd", "quant_pa", "decode_pa"])
+                                  "bsnd_n3_padded_heads", "quant_tnd", "quant_pa", "decode_pa",
+                                  "int8_tnd_fp16", "int8_pa_fp32"])
 def test_exact_integer_parity(name):
     """Small-integer inputs: every product and sum is exact in fp32, so the GPU
     must reproduce the oracle exactly, ties broken toward the lower index."""
@@ -99,12 +106,28 @@ def test_exact_integer_parity(name):
     if p.quant:
         for key in ("q_scale", "k_scale"):
             e = torch.randint(-2, 3, inp[key].shape, generator=g).to(torch.float32)
-            inp[key] = torch.pow(2.0, e)
+            inp[key] = torch.pow(2.0, e).to(inp[key].dtype)
     gi, gv, flags = run_gpu(p, inp)
     assert flags == 0
     o = oracle.run(p, inp)
     np.testing.assert_array_equal(gi, o["idx"])
     np.testing.assert_array_equal(gv, o["val"])
+
+
+def test_quant_int8_readme_example_full():
+    """The VllmQuantLightningIndexer README's A3 call: int8 q/k over the full
+    int8 range (|q.k| up to 2^21), fp16 scales and weights, PA keys."""
+    p, inp = synth.make_quant_int8_pa()
+    gi, gv, flags = run_gpu(p, inp)
+    assert flags == 0
+    check_against_oracle(p, inp, gi, gv)
+
+
+def test_quant_int8_varlen_sampled():
+    p, inp = synth.make_quant_varlen_int8(return_value=1)
+    gi, gv, flags = run_gpu(p, inp)
+    assert flags == 0
+    check_against_oracle(p, inp, gi, gv, rows=sample_rows(p, n_random=64, edge=16))
 
 
 def test_tiny_workload():

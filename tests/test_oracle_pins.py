@@ -67,6 +67,10 @@ CASES = [
     dict(layout_q="BSND", layout_k="PA_BSND", sparse_mode=3, quant=True, dtype_w="fp32",
          block_size=16),
     dict(layout_q="BSND", layout_k="BSND", sparse_mode=3, empty_rows=True),
+    dict(layout_q="TND", layout_k="TND", sparse_mode=3, quant=True, quant_dtype="int8",
+         dtype_scale="fp16", dtype_w="fp16"),
+    dict(layout_q="BSND", layout_k="PA_BSND", sparse_mode=0, quant=True, quant_dtype="int8",
+         dtype_w="fp32", block_size=16),
 ]
 
 
@@ -323,6 +327,36 @@ def test_quant_unit_scales_equal_plain_path():
     o2 = oracle.run(p2, inp2)
     np.testing.assert_array_equal(o["idx"], o2["idx"])
     np.testing.assert_array_equal(o["v64"], o2["v64"])
+
+
+def test_quant_int8_unit_scales_equal_plain_path():
+    p, inp = small(52, layout_q="BSND", layout_k="PA_BSND", sparse_mode=3, quant=True,
+                   quant_dtype="int8", dtype_scale="fp16", dtype_w="fp16", block_size=16)
+    inp = dict(inp)
+    inp["q_scale"] = torch.ones_like(inp["q_scale"])
+    inp["k_scale"] = torch.ones_like(inp["k_scale"])
+    o = oracle.run(p, inp)
+    # every int8 value is an integer of magnitude <= 128, exact in bf16
+    p2 = synth.Problem(**{**p.__dict__, "quant": False, "dtype_qk": "bf16"})
+    inp2 = dict(inp)
+    inp2["query"] = inp["query"].to(torch.float32).to(torch.bfloat16)
+    inp2["key"] = inp["key"].to(torch.float32).to(torch.bfloat16)
+    o2 = oracle.run(p2, inp2)
+    np.testing.assert_array_equal(o["idx"], o2["idx"])
+    np.testing.assert_array_equal(o["v64"], o2["v64"])
+
+
+def test_int8_quantizer_round_trip():
+    """The int8 input recipe: codes are round-half-even(x / (absmax/127)),
+    so code * scale is within half a step of x and the row's absmax maps to
+    +-127."""
+    g = torch.Generator().manual_seed(3)
+    x = torch.randn(50, 4, 16, generator=g)
+    codes, scale = synth.quantize_int8_per_row(x)
+    assert codes.dtype == torch.int8
+    back = codes.to(torch.float32) * scale.unsqueeze(-1)
+    assert torch.all((back - x).abs() <= 0.5 * scale.unsqueeze(-1) * (1 + 1e-6))
+    assert torch.all(codes.abs().to(torch.int32).amax(-1) == 127)
 
 
 def test_quant_power_of_two_scale_equivariance():

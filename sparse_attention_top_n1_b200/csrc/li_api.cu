@@ -151,6 +151,8 @@ WorkspaceLayout make_layout(const li_params &p, const Tiling &t)
     off += align_up(sizeof(BatchInfo) * (size_t)p.B, kAlign);
     w.blocks = off;
     off += align_up(sizeof(BlockInfo) * (size_t)w.max_blocks, kAlign);
+    w.starts = off;
+    off += align_up(sizeof(int4) * (size_t)kMaxScoreGrid, kAlign);
     w.scores = off;
     off += align_up(sizeof(float) * (size_t)w.rows * (size_t)w.ld, kAlign);
     w.total = off;
@@ -251,6 +253,7 @@ li_status run(const li_params *pp, bool quant, const void *query, const void *ke
         return fail(LI_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, w.total);
     const int sms = num_sms();
     if (sms <= 0) return fail(LI_ERR_CUDA, "no CUDA device");
+    if (sms > kMaxScoreGrid) return fail(LI_ERR_CUDA, "more than %d SMs", kMaxScoreGrid);
 
     const int es = elem_bytes(p.dtype_qk);
     const int inner = 128 / es;
@@ -331,6 +334,8 @@ li_status run(const li_params *pp, bool quant, const void *query, const void *ke
     pa.T1 = p.T1;
     pa.T2 = p.T2;
     pa.nq = t.nq;
+    pa.cta_start = reinterpret_cast<int4 *>(ws + w.starts);
+    pa.grid = sms;
     pa.max_blocks = w.max_blocks;
     pa.ld = w.ld;
     pa.pa_capacity = (int64_t)p.max_blocks_per_seq * p.block_size;
@@ -347,6 +352,7 @@ li_status run(const li_params *pp, bool quant, const void *query, const void *ke
     sa.block_table = block_table;
     sa.batches = batches;
     sa.blocks = blocks;
+    sa.cta_start = reinterpret_cast<const int4 *>(ws + w.starts);
     sa.hdr = hdr;
     sa.scores = scores;
     sa.ld = w.ld;

@@ -20,6 +20,7 @@ constexpr int kScoreThreads = 32 * (2 + kEpiWarps);
 constexpr int kTopkThreads = 512;
 constexpr int kPlanThreads = 1024;
 constexpr size_t kAlign = 256;
+constexpr int kMaxScoreGrid = 1024;   // score CTAs whose start the scheduler records
 constexpr int64_t kDefaultTimeoutNs = 2000000000LL;   // 2 s per pipeline wait
 
 // Per-batch sequence bookkeeping, clamped to what the tensors can hold.
@@ -52,7 +53,7 @@ struct PlanHeader {
 
 // Workspace carve-up (all offsets 256-byte aligned).
 struct WorkspaceLayout {
-    size_t header, batches, blocks, scores, total;
+    size_t header, batches, blocks, starts, scores, total;
     int64_t ld;           // floats per score row
     int64_t rows;         // query rows
     int32_t max_blocks;   // capacity of the block table
@@ -77,6 +78,8 @@ struct PlanArgs {
     int32_t nq, max_blocks;
     int64_t ld;            // score row capacity: key lengths are clamped to it
     int64_t pa_capacity;   // max_blocks_per_seq * block_size
+    int4 *cta_start;       // per score CTA: (block, tile, block's unit_start, block's ntiles)
+    int32_t grid;          // score CTAs
 };
 
 struct ScoreArgs {
@@ -86,6 +89,7 @@ struct ScoreArgs {
     const int32_t *block_table;
     const BatchInfo *batches;
     const BlockInfo *blocks;
+    const int4 *cta_start;      // where each CTA's share of the work list begins
     PlanHeader *hdr;
     float *scores;
     int64_t ld;

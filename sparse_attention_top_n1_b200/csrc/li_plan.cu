@@ -12,6 +12,9 @@
 //   BlockInfo[g]  query block g: its batch, first query, the number of key
 //                 tiles its last (most-seeing) query needs, and its first
 //                 position in the weighted work list (tiles + kQCost per block)
+//   cta_start[c]  where score CTA c's equal share of the work list begins:
+//                 its first block, tile, and that block's unit_start and
+//                 tile count (one load for the CTA instead of a search)
 //   PlanHeader    totals and the device status word (cleared here: this is
 //                 the first kernel of every call)
 // Lengths outside what the tensors or the declared bounds can hold are
@@ -58,6 +61,7 @@ __device__ int32_t block_inclusive_scan(int32_t &v, int32_t *tmp)
 }
 
 constexpr int kSmemBatches = 1024;      // batches mirrored in shared memory
+constexpr int kSmemBlocks = 8192;       // query blocks whose first unit is mirrored
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a)
 {
@@ -65,6 +69,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a)
     __shared__ int32_t s_flags;
     __shared__ int32_t s_blk_off[kSmemBatches];
     __shared__ int2 s_len[kSmemBatches];          // (Sq, Sk)
+    __shared__ int32_t s_ustart[kSmemBlocks];     // unit_start of block g
     const bool in_smem = a.B <= kSmemBatches;
     const int tid = threadIdx.x;
     if (tid == 0) s_flags = 0;
@@ -184,8 +189,39 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a)
         if (g < total_blocks) {
             blk.unit_start = carry + incl - weight;
             a.blocks[g] = blk;
+            if (g < kSmemBlocks) s_ustart[g] = blk.unit_start;
         }
         carry += tot;
+    }
+
+    // 3. the start of every score CTA's share [total*c/grid, total*(c+1)/grid)
+    //    of the work list: the last block whose first unit is at or before
+    //    the share's first unit w0, and the tile of w0 inside it.  Blocks
+    //    without tiles share their first unit with the next block, so the
+    //    last such block always has the tile (w0 < its end, or the next block
+    //    would start at or before w0).
+    const int32_t total_units = carry;
+    __syncthreads();   // s_ustart and blocks[] visible to the whole CTA
+    const bool ustart_in_smem = total_blocks <= kSmemBlocks;
+    for (int c = tid; c < a.grid; c += kPlanThreads) {
+        int4 st = make_int4(0, 0, 0, 0);
+        if (total_blocks > 0 && total_units > 0) {
+            const int32_t w0 = (int32_t)(((int64_t)total_units * c) / a.grid);
+            int lo = 0, hi = total_blocks - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                const int32_t u = ustart_in_smem ? s_ustart[mid] : a.blocks[mid].unit_start;
+                if (u <= w0) lo = mid; else hi = mid - 1;
+            }
+            const int32_t u0 = ustart_in_smem ? s_ustart[lo] : a.blocks[lo].unit_start;
+            const int32_t u1 = lo + 1 < total_blocks
+                                   ? (ustart_in_smem ? s_ustart[lo + 1] : a.blocks[lo + 1].unit_start)
+                                   : total_units;
+            int32_t tile = w0 - u0 - kQCost;
+            if (tile < 0) tile = 0;
+            st = make_int4(lo, tile, u0, u1 - u0 - kQCost);
+        }
+        a.cta_start[c] = st;
     }
     if (tid == 0) {
         a.hdr->total_blocks = total_blocks;

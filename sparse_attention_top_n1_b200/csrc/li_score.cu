@@ -75,19 +75,16 @@ struct Walker {
             load_block();
         }
     }
-    __device__ void init(int w0, int w1)
+    // start at the scheduler's record of where this CTA's share [w0, w1)
+    // begins: the last block starting at or before w0, the tile inside it,
+    // moved past blocks without a tile in the share
+    __device__ void init_from(const int4 st, int w1)
     {
         w_end = w1;
-        int lo = 0, hi = nblocks - 1;                  // last block starting at or before w0
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (blocks[mid].unit_start <= w0) lo = mid; else hi = mid - 1;
-        }
-        qb = lo;
-        load_block();
-        tile = w0 - start - kQCost;
-        if (tile < 0) tile = 0;
-        normalize();
+        qb = st.x;
+        tile = st.y;
+        start = st.z;
+        ntiles = st.w;
     }
     __device__ bool valid() const { return qb < nblocks && start + kQCost + tile < w_end; }
     __device__ void next()
@@ -333,7 +330,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         // global loads on the copy path.
         if (w_begin < w_end && nblocks > 0) {
             Walker w{a.blocks, nblocks, 0, 0, 0, 0, 0};
-            w.init(w_begin, w_end);
+            w.init_from(a.cta_start[blockIdx.x], w_end);
             int stage = 0, prev_qb = -1;
             uint32_t phase = 0, qphase = 0;
             uint32_t armed = 0, par = 0, q_armed = 0, q_par = 0;
@@ -455,7 +452,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0 && w_begin < w_end && nblocks > 0) {
             Walker w{a.blocks, nblocks, 0, 0, 0, 0, 0};
-            w.init(w_begin, w_end);
+            w.init_from(a.cta_start[blockIdx.x], w_end);
             int stage = 0, acc = 0, prev_qb = -1;
             uint32_t phase = 0, acc_phase = 0, qphase = 0, idesc = 0;
             bool issued = false;
@@ -530,7 +527,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         float *myW = sW + ew * 128;
         if (w_begin < w_end && nblocks > 0) {
             Walker w{a.blocks, nblocks, 0, 0, 0, 0, 0};
-            w.init(w_begin, w_end);
+            w.init_from(a.cta_start[blockIdx.x], w_end);
             int acc = 0, prev_qb = -1, nchunks = 0;
             uint32_t acc_phase = 0;
             BlockInfo blk{};

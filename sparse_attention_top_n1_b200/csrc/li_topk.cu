@@ -5,21 +5,28 @@
 // read as: value descending, ties by lower key index; slots past the number
 // of candidates hold -1 / -inf ("通用约束").
 //
-// One CTA of 512 threads per row:
-//   1. Radix select.  Scores are mapped to order-preserving uint32 keys
-//      (-0.0 is first folded into +0.0).  Three histogram passes over the row
-//      (11, 11 and 10 bits, most significant first) find the exact key T of
-//      the k-th largest element and how many of the k must be taken from the
-//      elements equal to T.
+// Rows of up to 16384 keys: one CTA of 512 threads per row.
+//   The row is cached in shared memory as order-preserving uint32 keys
+//   (-0.0 folded into +0.0).  The bucket path histograms it over 2048 linear
+//   value buckets between its min and max, finds the bucket holding the k-th
+//   largest value, scatters the selected keys grouped by bucket, and gives
+//   each its final slot: its bucket's offset plus its rank inside the bucket,
+//   counted by (value desc, index asc).  When a bucket is too full for
+//   counting (ties, clustered values) or the range is degenerate, the exact
+//   radix path runs instead:
+//   1. Radix select: three histogram passes (11, 11 and 10 bits, most
+//      significant first) find the exact key T of the k-th largest element
+//      and how many of the k come from the elements equal to T.
 //   2. Compaction in index order: every key > T, plus the lowest-index keys
-//      == T, written to a buffer in ascending index order.
-//   3. A stable LSB radix sort of the selected keys by descending value (4
-//      passes of 8 bits; a pass whose digit is the same for every selected
-//      key is skipped).  Stability keeps equal values in index order.
+//      == T.
+//   3. A stable LSB radix sort by descending value (4 passes of 8 bits; a
+//      pass whose digit is the same for every selected key is skipped).
 //   4. Write indices and values, pad with -1 / -inf.
-// Rows of up to `cap` elements are cached in shared memory; longer rows are
-// streamed from global memory (L2) on every pass.
+// Longer rows (decode over long contexts): a thread-block cluster of 8 CTAs
+// per row runs the bucket method over distributed shared memory (see the
+// long-rows section below).
 #include <cstdint>
+#include <cooperative_groups.h>
 
 #include "li_internal.cuh"
 #include "ptx.cuh"
@@ -27,9 +34,7 @@
 namespace li {
 namespace {
 
-constexpr int kWarps = kTopkThreads / 32;
-constexpr int kSortMaxRounds = 2048 / (kWarps * 32);   // rounds of 32 per warp for kmax <= 2048
-static_assert(kWarps * 256 <= 4096, "per-warp radix counters must fit the 4096-word histogram");
+constexpr int kMaxWarps = 16;        // CTAs have at most 512 threads
 
 __device__ __forceinline__ uint32_t to_key(float f)
 {
@@ -51,11 +56,12 @@ __device__ __forceinline__ uint32_t lanemask_lt()
     return m;
 }
 
-// Exclusive scan of one value per thread over the whole CTA; also returns the
-// total.  `tmp` holds kWarps + 1 ints.  Contains __syncthreads.
-template <typename T>
+// Exclusive scan of one value per thread over the whole CTA of NT threads;
+// also returns the total.  `tmp` holds NT/32 + 1 values.  Contains __syncthreads.
+template <int NT, typename T>
 __device__ __forceinline__ T block_exclusive_scan(T v, T *tmp, T &total)
 {
+    constexpr int kWarps = NT / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     T x = v;
 #pragma unroll
@@ -132,19 +138,27 @@ struct TopkSmem {
     uint32_t *cache;    // the row as keys, when it fits
 };
 
+constexpr int kMaxCluster = 8;       // CTAs per row for the longest rows
+
 struct TopkShared {
-    uint32_t tmp32[kWarps + 1];
-    uint64_t tmp64[kWarps + 1];
+    uint32_t tmp32[kMaxWarps + 1];
+    uint64_t tmp64[kMaxWarps + 1];
     uint32_t digit, above, vor, vand, kmin, kmax, maxbin;
+    uint32_t pmin[kMaxCluster], pmax[kMaxCluster];   // slice ranges pushed by the cluster
+    uint32_t verdict;                                // CTA 0 -> all: bucket method taken
+    uint32_t bstar, above_b;                         // CTA 0 -> all: threshold bucket
 };
 
 // ---------------------------------------------------------------- radix path
 // Exact for every input (ties, equal values, any range): three histogram
 // passes find the k-th key, an index-order compaction selects, a stable LSB
 // radix sort orders.  Used when the bucket path declines a row.
+template <int NT>
 __device__ void radix_topk(const RowSrc &src, int n, int k, int m, const TopkSmem &s,
                            TopkShared &sh, int32_t *oidx, float *oval)
 {
+    constexpr int kTopkThreads = NT, kWarps = NT / 32;
+    constexpr int kSortMaxRounds = 2048 / NT;       // rounds of 32 per warp for kmax <= 2048
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int n4 = (n + 3) >> 2;
     uint32_t *hist = s.hist, *keyA = s.keyA, *keyB = s.keyB;
@@ -190,7 +204,7 @@ __device__ void radix_topk(const RowSrc &src, int n, int k, int m, const TopkSme
             uint32_t c = 0;
             for (int e = 0; e < per; ++e) c += hist[bins - 1 - (tid * per + e)];
             uint32_t tot;
-            uint32_t above = block_exclusive_scan<uint32_t>(c, s_tmp32, tot);
+            uint32_t above = block_exclusive_scan<NT, uint32_t>(c, s_tmp32, tot);
             if (above < (uint32_t)remaining && above + c >= (uint32_t)remaining) {
                 uint32_t acc = above;
                 for (int e = 0; e < per; ++e) {
@@ -241,7 +255,7 @@ __device__ void radix_topk(const RowSrc &src, int n, int k, int m, const TopkSme
                 }
             }
             uint64_t packed = ((uint64_t)neq << 32) | ngt, tot;
-            uint64_t before = block_exclusive_scan<uint64_t>(packed, s_tmp64, tot);
+            uint64_t before = block_exclusive_scan<NT, uint64_t>(packed, s_tmp64, tot);
             uint32_t gt_b = gt_carry + (uint32_t)before;
             uint32_t eq_b = eq_carry + (uint32_t)(before >> 32);
             if (j4 < n4) {
@@ -315,7 +329,7 @@ __device__ void radix_topk(const RowSrc &src, int n, int k, int m, const TopkSme
                 sum += own[j];
             }
             uint32_t tot;
-            uint32_t off = block_exclusive_scan<uint32_t>(sum, s_tmp32, tot);
+            uint32_t off = block_exclusive_scan<NT, uint32_t>(sum, s_tmp32, tot);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int c = tid * 8 + j, d = c / kWarps, wi = c % kWarps;
@@ -352,7 +366,6 @@ __device__ void radix_topk(const RowSrc &src, int n, int k, int m, const TopkSme
         }
     }
 }
-
 
 // ---------------------------------------------------------------- bucket path
 // Linear value buckets over [min, max] of the row (monotone in the value):
@@ -402,7 +415,7 @@ __device__ bool bucket_topk(const RowSrc &src, int n, int k, int m, int kmax, co
 #pragma unroll
     for (int e = 0; e < per; ++e) c += hist[kBuckets - 1 - (tid * per + e)];
     uint32_t tot;
-    const uint32_t above_t = block_exclusive_scan<uint32_t>(c, sh.tmp32, tot);
+    const uint32_t above_t = block_exclusive_scan<kTopkThreads, uint32_t>(c, sh.tmp32, tot);
     uint32_t acc = above_t;
 #pragma unroll
     for (int e = 0; e < per; ++e) {
@@ -588,7 +601,330 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a)
     __syncthreads();
 
     if (!bucket_topk(src, n, k, m, a.kmax, s, sh, oidx, oval))
-        radix_topk(src, n, k, m, s, sh, oidx, oval);
+        radix_topk<kTopkThreads>(src, n, k, m, s, sh, oidx, oval);
+}
+
+// Number of candidate keys of a row: the visible prefix of the batch's keys
+// (indexer mode) or row_len[row] (standalone mode).
+__device__ __forceinline__ int row_length(const TopkArgs &a, int row)
+{
+    if (a.standalone) {
+        const int n = a.row_len ? a.row_len[row] : (int)a.ld;
+        return n < 0 ? 0 : (n > a.ld ? (int)a.ld : n);
+    }
+    int b, i;
+    if (a.layout_q == LI_BSND) {
+        b = row / a.S1;
+        i = row % a.S1;
+    } else {
+        int lo = 0, hi = a.B - 1;                   // last batch with q_off <= row
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (a.batches[mid].q_off <= row) lo = mid; else hi = mid - 1;
+        }
+        b = lo;
+        i = row - a.batches[b].q_off;
+    }
+    const BatchInfo bi = a.batches[b];
+    if (i < 0 || i >= bi.Sq) return 0;
+    if (a.mode != 3) return bi.Sk;
+    const int lim = i + 1 + bi.Sk - bi.Sq;
+    return lim < 0 ? 0 : (lim < bi.Sk ? lim : bi.Sk);
+}
+
+template <int NT>
+__device__ __forceinline__ void pad_row(int32_t *oidx, float *oval, int from, int k)
+{
+    for (int j = from + (int)threadIdx.x; j < k; j += NT) {
+        oidx[j] = -1;
+        if (oval) oval[j] = __uint_as_float(0xFF800000u);
+    }
+}
+
+// Barrier over the whole cluster (C > 1) or the CTA.  A cluster barrier
+// orders the shared-memory writes of every CTA before the reads after it.
+template <int C>
+__device__ __forceinline__ void csync()
+{
+    if constexpr (C > 1) cooperative_groups::this_cluster().sync();
+    else __syncthreads();
+}
+
+// The same shared-memory object in CTA `rank` of this cluster.
+template <int C, typename T>
+__device__ __forceinline__ T *peer(T *p, int rank)
+{
+    if constexpr (C > 1) return cooperative_groups::this_cluster().map_shared_rank(p, rank);
+    else return p;
+}
+
+// ---------------------------------------------------------------- long rows
+// Rows longer than one CTA caches (decode over long contexts) are split over a
+// thread-block cluster of C CTAs, CTA r owning the r-th slice of the row.  The
+// bucket method runs cluster-wide through distributed shared memory:
+//   1. every CTA pushes its slice's min/max to all CTAs of the cluster;
+//   2. every CTA histograms its slice over kCBuckets linear value buckets and
+//      adds the counts into CTA 0;
+//   3. CTA 0 scans the buckets from the top, finds the bucket holding the
+//      m-th largest value and broadcasts it (or declines, as the one-CTA
+//      bucket path does);
+//   4. every CTA reserves room in CTA 0 bucket by bucket and scatters its
+//      selected keys there;
+//   5. CTA 0 ranks each key inside its bucket and writes the row.
+// A declined row is done by CTA 0 with the exact radix method, streamed.
+constexpr int kCBuckets = 4096;
+
+// One row per cluster of C CTAs of NT threads; each thread holds up to EPT
+// scores of its CTA's slice in registers (float4 group g of thread t covers
+// slice keys 4*(t + g*NT) .. +3).  Selected keys travel as one 64-bit word,
+// (order-preserving key << 32) | ~index, so that a larger word means a larger
+// value or, for equal values, a lower index.
+template <int C, int NT, int EPT>
+__global__ void __launch_bounds__(NT) topk_cluster_kernel(TopkArgs a)
+{
+    constexpr int G = EPT / 4;                  // float4 groups per thread
+    constexpr int PER_T = kCBuckets / NT;        // buckets per thread in the scan
+    extern __shared__ __align__(16) uint8_t smem[];
+    __shared__ TopkShared sh;
+
+    const int tid = threadIdx.x;
+    int rank = 0;
+    if constexpr (C > 1) rank = (int)cooperative_groups::this_cluster().block_rank();
+    const int row = blockIdx.x / C;
+    const int k = a.k;
+    grid_dependency_wait();             // the score rows come from the previous kernel
+
+    const int n = row_length(a, row);
+    int32_t *oidx = a.out_idx + (int64_t)row * k;
+    float *oval = a.out_val ? a.out_val + (int64_t)row * k : nullptr;
+    const int m = n < k ? n : k;
+    if (m == 0) {                       // the same in every CTA of the cluster
+        if (rank == 0) pad_row<NT>(oidx, oval, 0, k);
+        return;
+    }
+
+    // shared memory: bucket counts | bucket cursors | selected words | their
+    // buckets | tail (candidates + row counts, or the radix sort's buffer)
+    uint32_t *hist = reinterpret_cast<uint32_t *>(smem);
+    uint32_t *cur = hist + kCBuckets;
+    uint64_t *sel = reinterpret_cast<uint64_t *>(cur + kCBuckets);
+    uint16_t *selb = reinterpret_cast<uint16_t *>(sel + a.kmax);
+    uint32_t *tail = reinterpret_cast<uint32_t *>(selb + a.kmax);
+    uint64_t *cand = reinterpret_cast<uint64_t *>(tail);
+    uint32_t *gcnt = tail + 2 * kCandLimit;
+
+    const float *grow = a.scores + (int64_t)row * a.ld;
+    // whole row with the exact radix method, streamed from global memory (CTA 0)
+    auto radix_row = [&]() {
+        TopkSmem s;
+        s.hist = hist;
+        s.keyA = reinterpret_cast<uint32_t *>(sel);
+        s.idxA = reinterpret_cast<int32_t *>(s.keyA + a.kmax);
+        s.keyB = tail;
+        s.idxB = reinterpret_cast<int32_t *>(tail + a.kmax);
+        RowSrc full;
+        full.g = grow;
+        full.c = nullptr;
+        full.n = n;
+        radix_topk<NT>(full, n, k, m, s, sh, oidx, oval);
+    };
+    if (n > C * NT * EPT) {             // longer than the registers hold
+        if (rank == 0) radix_row();
+        return;
+    }
+
+    // this CTA's slice [lo, hi) of the row; lo is a multiple of 4
+    const int per = (((n + C - 1) / C) + 3) & ~3;
+    const int lo = min(n, rank * per), hi = min(n, lo + per);
+    const int len = hi - lo;
+    const int n4 = (len + 3) >> 2;
+
+    // ---- 1. the slice into registers; push its range to the cluster
+    if (tid == 0) {
+        sh.kmin = 0xFFFFFFFFu;
+        sh.kmax = 0u;
+        sh.maxbin = 0u;
+    }
+    for (int j = tid; j < kCBuckets; j += NT) hist[j] = 0;
+    if (C > 1 && rank == 0)
+        for (int j = tid; j < kCBuckets; j += NT) gcnt[j] = 0;
+    float v[G][4];
+    {
+        const float4 *g4 = reinterpret_cast<const float4 *>(grow + lo);
+        float lmin = __int_as_float(0x7F800000), lmax = __int_as_float(0xFF800000);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const int j4 = tid + g * NT;
+            if (j4 < n4) {
+                const float4 x = g4[j4];
+                v[g][0] = x.x;
+                v[g][1] = x.y;
+                v[g][2] = x.z;
+                v[g][3] = x.w;
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (j4 * 4 + e < len) {
+                        lmin = fminf(lmin, v[g][e]);
+                        lmax = fmaxf(lmax, v[g][e]);
+                    }
+            }
+        }
+        // NaN scores are skipped by fminf / fmaxf; their order is unspecified
+        uint32_t kmn = to_key(lmin), kmx = to_key(lmax);
+        kmn = warp_min(kmn);
+        kmx = warp_max(kmx);
+        __syncthreads();                // sh initialised
+        if ((tid & 31) == 0) {          // one shared atomic per warp, not per thread
+            atomicMin(&sh.kmin, kmn);
+            atomicMax(&sh.kmax, kmx);
+        }
+    }
+    __syncthreads();
+    if (tid < C) {                      // thread r tells CTA r this slice's range
+        TopkShared *ps = peer<C>(&sh, tid);
+        ps->pmin[rank] = sh.kmin;
+        ps->pmax[rank] = sh.kmax;
+    }
+    csync<C>();                         // S1: ranges pushed, counts cleared
+
+    uint32_t kmin = sh.pmin[0], kmax = sh.pmax[0];
+#pragma unroll
+    for (int r = 1; r < C; ++r) {
+        kmin = min(kmin, sh.pmin[r]);
+        kmax = max(kmax, sh.pmax[r]);
+    }
+    const float fmin = from_key(kmin), fmax = from_key(kmax);
+    const float range = fmax - fmin;
+    const float scale = (float)kCBuckets / range;
+    const float boff = -fmin * scale;
+    if (!(range > 0.f) || !isfinite(range) || !isfinite(scale) || !isfinite(boff)) {
+        if (rank == 0) radix_row();     // one value, or non-finite scores
+        return;
+    }
+    // bucket of a score: floor(x * scale + boff), clamped; monotone in x
+    auto bucket = [&](float x) {
+        const int b = __float2int_rz(fmaf(x, scale, boff));
+        return b < 0 ? 0 : (b >= kCBuckets ? kCBuckets - 1 : b);
+    };
+
+    // ---- 2. histogram of the slice; CTA 0 gathers the row's counts
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+        if (tid + g * NT < n4)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if ((tid + g * NT) * 4 + e < len) atomicAdd(&hist[bucket(v[g][e])], 1u);
+    uint32_t *gc = hist;                // the row's counts (one CTA: its own)
+    if constexpr (C > 1) {
+        __syncthreads();
+        uint32_t *g0 = peer<C>(gcnt, 0);
+        for (int j = tid; j < kCBuckets; j += NT)
+            if (hist[j]) atomicAdd(&g0[j], hist[j]);
+        gc = gcnt;                      // meaningful in CTA 0
+    }
+    csync<C>();                         // S2: CTA 0 holds the row's counts
+
+    // ---- 3. CTA 0: threshold bucket, bucket offsets and the verdict
+    if (rank == 0) {
+        // thread t owns buckets kCBuckets-1-(t*PER_T+e), counted from the top;
+        // a bucket lies wholly above the threshold iff its end offset < m
+        uint32_t c = 0;
+#pragma unroll
+        for (int e = 0; e < PER_T; ++e) c += gc[kCBuckets - 1 - (tid * PER_T + e)];
+        uint32_t tot;
+        uint32_t acc = block_exclusive_scan<NT, uint32_t>(c, sh.tmp32, tot);
+        uint32_t lm = 0;
+#pragma unroll
+        for (int e = 0; e < PER_T; ++e) {
+            const int d = kCBuckets - 1 - (tid * PER_T + e);
+            const uint32_t h = gc[d];
+            if (acc < (uint32_t)m && acc + h >= (uint32_t)m) {
+                sh.digit = (uint32_t)d;
+                sh.above = acc;
+            }
+            if (acc + h < (uint32_t)m) lm = max(lm, h);
+            cur[d] = acc;               // first output slot of bucket d
+            acc += h;
+        }
+        lm = warp_max(lm);
+        if ((tid & 31) == 0 && lm) atomicMax(&sh.maxbin, lm);
+        __syncthreads();
+        if (tid < C) {                  // thread r tells CTA r
+            TopkShared *ps = peer<C>(&sh, tid);
+            ps->verdict = (sh.maxbin <= (uint32_t)kBinLimit && gc[sh.digit] <= (uint32_t)kCandLimit) ? 1u : 0u;
+            ps->bstar = sh.digit;
+            ps->above_b = sh.above;
+        }
+    }
+    csync<C>();                         // S3: every CTA knows the verdict
+    if (!sh.verdict) {
+        if (rank == 0) radix_row();     // a bucket too full for counting
+        return;
+    }
+
+    // ---- 4. scatter the selected words into CTA 0, grouped by bucket; the
+    //         threshold bucket's words into its candidate list
+    const int bstar = (int)sh.bstar;
+    const uint32_t above = sh.above_b;
+    uint64_t *sel0 = peer<C>(sel, 0), *cand0 = peer<C>(cand, 0);
+    uint16_t *selb0 = peer<C>(selb, 0);
+    uint32_t *slot = cur;               // one CTA: the bucket cursors themselves
+    if constexpr (C > 1) {
+        // reserve this slice's share of every bucket from the threshold up;
+        // its counts become its own cursors
+        uint32_t *cur0 = peer<C>(cur, 0);
+        for (int j = tid; j < kCBuckets; j += NT) {
+            const uint32_t h = hist[j];
+            if (j >= bstar && h) hist[j] = atomicAdd(&cur0[j], h);
+        }
+        __syncthreads();
+        slot = hist;
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+        if (tid + g * NT < n4)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int j = (tid + g * NT) * 4 + e;
+                if (j < len) {
+                    const int b = bucket(v[g][e]);
+                    if (b >= bstar) {
+                        const uint32_t pos = atomicAdd(&slot[b], 1u);
+                        const uint64_t w = ((uint64_t)to_key(v[g][e]) << 32) | (uint32_t)~(uint32_t)(lo + j);
+                        if (b > bstar) {
+                            sel0[pos] = w;
+                            selb0[pos] = (uint16_t)b;
+                        } else {
+                            cand0[pos - above] = w;
+                        }
+                    }
+                }
+            }
+    csync<C>();                         // S4: every selected word is in CTA 0
+    if (rank != 0) return;
+
+    // ---- 5. CTA 0: rank inside the buckets and write
+    auto emit = [&](uint32_t pos, uint64_t w) {
+        oidx[pos] = (int32_t)~(uint32_t)w;
+        if (oval) oval[pos] = from_key((uint32_t)(w >> 32));
+    };
+    const uint32_t cstar = gc[bstar];
+    const uint32_t need = (uint32_t)m - above;
+    for (uint32_t e = tid; e < cstar; e += NT) {
+        const uint64_t w = cand[e];
+        uint32_t r = 0;
+        for (uint32_t q = 0; q < cstar; ++q) r += cand[q] > w;
+        if (r < need) emit(above + r, w);
+    }
+    for (uint32_t p = tid; p < above; p += NT) {
+        const uint64_t w = sel[p];
+        const int b = selb[p];
+        const uint32_t cnt = gc[b], s0 = cur[b] - cnt;   // the cursor ended one bucket past
+        uint32_t r = 0;
+        for (uint32_t q = s0; q < s0 + cnt; ++q) r += sel[q] > w;
+        emit(s0 + r, w);
+    }
+    pad_row<NT>(oidx, oval, m, k);
 }
 
 }  // namespace
@@ -600,7 +936,7 @@ size_t topk_smem_bytes(int cap, int kmax)
            (cache > pingpong ? cache : pingpong);
 }
 
-cudaError_t launch_topk(const TopkArgs &a, cudaStream_t s)
+cudaError_t launch_single(const TopkArgs &a, cudaStream_t s)
 {
     const size_t smem = topk_smem_bytes(a.cap, a.kmax);
     cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -618,6 +954,53 @@ cudaError_t launch_topk(const TopkArgs &a, cudaStream_t s)
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, topk_kernel, a);
+}
+
+// Shared memory of one cluster CTA: bucket counts and cursors, the selected
+// words and their buckets, and a tail for the candidates and row counts (or
+// the radix sort's second buffer).
+size_t topk_cluster_smem_bytes(int kmax)
+{
+    const size_t tail_bucket = (size_t)2 * kCandLimit + kCBuckets, tail_radix = (size_t)2 * kmax;
+    return (size_t)2 * kCBuckets * 4 + (size_t)kmax * 10 +
+           (tail_bucket > tail_radix ? tail_bucket : tail_radix) * 4;
+}
+
+template <int EPT>
+cudaError_t launch_cluster(const TopkArgs &a, cudaStream_t s)
+{
+    auto kern = topk_cluster_kernel<kMaxCluster, kTopkThreads, EPT>;
+    const size_t smem = topk_cluster_smem_bytes(a.kmax);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)a.rows * kMaxCluster);
+    cfg.blockDim = dim3(kTopkThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = a.standalone ? 0 : 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = kMaxCluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+// Rows that fit one CTA's cache (ld <= a.cap) take one CTA each; longer rows
+// a cluster of kMaxCluster CTAs whose threads hold EPT keys each (rows beyond
+// kMaxCluster * 512 * 32 keys take the cluster's streamed radix path).
+cudaError_t launch_topk(const TopkArgs &a, cudaStream_t s)
+{
+    if (a.rows <= 0) return cudaSuccess;
+    if (a.ld <= a.cap) return launch_single(a, s);
+    const int64_t per_thread = (a.ld + (int64_t)kMaxCluster * kTopkThreads - 1) / ((int64_t)kMaxCluster * kTopkThreads);
+    if (per_thread <= 8) return launch_cluster<8>(a, s);
+    if (per_thread <= 16) return launch_cluster<16>(a, s);
+    return launch_cluster<32>(a, s);
 }
 
 }  // namespace li

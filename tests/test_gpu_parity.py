@@ -188,12 +188,16 @@ def _topk_reference(rows_np, lens, k):
                                        (8192, 2048, "quarters"), (40000, 2048, "normal"),
                                        (40000, 512, "quarters"), (64, 100, "normal"),
                                        (4096, 1024, "levels"), (16384, 2048, "levels"),
-                                       (2048, 2048, "levels"), (5000, 700, "constant")])
+                                       (2048, 2048, "levels"), (5000, 700, "constant"),
+                                       (65536, 2048, "levels"), (70000, 1, "normal"),
+                                       (140000, 2048, "normal"), (20000, 2048, "constant")])
 def test_topk_stage_exact(ld, k, kind):
     """Exact against a lexsort reference.  'quarters' (values on a 0.25 grid,
     every 7th -0.0) and 'constant' rows force the radix fallback; 'levels'
     (~7 keys per distinct value) keeps the bucket path with ties inside and
-    at the threshold bucket."""
+    at the threshold bucket.  Rows longer than 16384 keys run on a cluster of
+    CTAs (bucket path, radix fallback, and beyond 131072 keys the streamed
+    radix path)."""
     g = torch.Generator().manual_seed(ld + k)
     R = 12
     x = torch.randn(R, ld, generator=g)

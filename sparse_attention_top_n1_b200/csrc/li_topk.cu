@@ -672,7 +672,7 @@ __device__ __forceinline__ T *peer(T *p, int rank)
 //      selected keys there;
 //   5. CTA 0 ranks each key inside its bucket and writes the row.
 // A declined row is done by CTA 0 with the exact radix method, streamed.
-constexpr int kCBuckets = 4096;
+constexpr int kCBuckets = 2048;      // 52 KB per CTA: the 512 CTAs of 64 long rows fit one wave
 
 // One row per cluster of C CTAs of NT threads; each thread holds up to EPT
 // scores of its CTA's slice in registers (float4 group g of thread t covers

@@ -42,6 +42,7 @@ class OrProblem(ctypes.Structure):
         ("key_block_stride", ctypes.c_int64),
         ("sparse_count", ctypes.c_int32), ("sparse_mode", ctypes.c_int32),
         ("return_value", ctypes.c_int32), ("mutation", ctypes.c_int32),
+        ("init_num", ctypes.c_int32), ("local_num", ctypes.c_int32),
     ]
 
 
@@ -101,7 +102,8 @@ def make_problem(p, mutation: int = 0) -> OrProblem:
         N2=p.N2, D=p.D, num_blocks=p.num_blocks, block_size=p.block_size,
         max_blocks_per_seq=p.max_blocks_per_seq, key_block_stride=p.key_block_stride,
         sparse_count=p.sparse_count, sparse_mode=p.sparse_mode,
-        return_value=p.return_value, mutation=mutation)
+        return_value=p.return_value, mutation=mutation,
+        init_num=getattr(p, "init_num", 0), local_num=getattr(p, "local_num", 0))
 
 
 def max_key_len(p, inputs) -> int:

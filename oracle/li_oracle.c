@@ -18,6 +18,12 @@
  *   Top-k: order the visible keys by s descending (ties: lower key index
  *   first), keep min(k, visible) of them, pad the rest with index -1 and value
  *   -inf (CANN guide, "通用约束": invalid slots are -1 / -inf).
+ *   Sink tokens and the local window (the open-sourcing issue's comparison of
+ *   the MT lightning_indexer, which lists init_num -- sink tokens always
+ *   selected -- and local_num -- the diagonal local window): the first
+ *   init_num and the last local_num visible keys are always kept; the other
+ *   min(k, visible) - |forced| slots take the best of the remaining visible
+ *   keys; all kept keys are then ordered as above.
  *
  * Everything is evaluated in double precision from the exact values the
  * stored bits encode (bf16, fp16, fp8 e4m3 and int8 are decoded here from
@@ -56,6 +62,7 @@ typedef struct {
     int64_t key_block_stride;      /* elements between PA blocks; 0 = block_size*N2*D */
     int32_t sparse_count, sparse_mode, return_value;
     int32_t mutation;              /* 0 = the real oracle; >0 plants one mistake */
+    int32_t init_num, local_num;   /* forced sink tokens / local window (0 = none) */
 } or_problem;
 
 /* ---- decoders, from the format definitions ------------------------------ */
@@ -318,6 +325,37 @@ int li_oracle_rows(const or_problem *p, const void *query, const void *key, cons
         else
             qsort(c, (size_t)nc, sizeof(cand), cmp_cand);
         int64_t keep = nc < kk ? nc : kk;
+        if (p->init_num > 0 || p->local_num > 0) {
+            /* visible keys are t in [0, nv): force t < init_num and t >= nv - local_num */
+            int64_t nv = 0;
+            for (int64_t t = 0; t < s.Sk; ++t)
+                if (visible(p, s, i, t)) ++nv;
+            cand *f = (cand *)malloc(sizeof(cand) * (size_t)(nc ? nc : 1));
+            cand *o = (cand *)malloc(sizeof(cand) * (size_t)(nc ? nc : 1));
+            if (!f || !o) {
+                bad |= 1;
+                free(f); free(o); free(c); free(qv); free(wv); free(sq); free(kv);
+                continue;
+            }
+            int64_t nf = 0, no = 0;
+            /* planted mistake 7: the local window one key short */
+            const int64_t lo_local = nv - p->local_num + (p->mutation == 7 ? 1 : 0);
+            for (int64_t j = 0; j < nc; ++j) {
+                const int forced = c[j].t < p->init_num || c[j].t >= lo_local;
+                if (forced) f[nf++] = c[j]; else o[no++] = c[j];
+            }
+            qsort(o, (size_t)no, sizeof(cand), cmp_cand);          /* the best others */
+            int64_t take = keep - nf;
+            if (take < 0) take = 0;
+            if (take > no) take = no;
+            for (int64_t j = 0; j < take; ++j) f[nf++] = o[j];
+            qsort(f, (size_t)nf, sizeof(cand), cmp_cand);          /* all kept, in order */
+            if (nf > keep) nf = keep;
+            memcpy(c, f, sizeof(cand) * (size_t)nf);
+            keep = nf;
+            free(f);
+            free(o);
+        }
         for (int64_t j = 0; j < keep; ++j) {
             oi[j] = (int32_t)c[j].t;
             ov[j] = (float)c[j].s;
@@ -329,4 +367,4 @@ int li_oracle_rows(const or_problem *p, const void *query, const void *key, cons
     return bad ? -1 : 0;
 }
 
-int li_oracle_abi_version(void) { return 1; }
+int li_oracle_abi_version(void) { return 2; }

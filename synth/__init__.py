@@ -75,6 +75,8 @@ class Problem:
     pre_tokens: int = INT64_MAX
     next_tokens: int = INT64_MAX
     max_seqlen_k: int = 0           # host-side bound on any key length (0 = derive)
+    init_num: int = 0               # sink tokens always selected (first visible keys)
+    local_num: int = 0              # local window always selected (last visible keys)
 
     @property
     def rows(self) -> int:
@@ -267,7 +269,7 @@ def make_random(seed: int, *, layout_q="BSND", layout_k="BSND", dtype_qk="bf16",
                 dtype_w="bf16", B=2, S1=40, S2=300, N1=8, D=128, sparse_count=64,
                 sparse_mode=3, return_value=1, ragged=True, block_size=64,
                 quant=False, empty_rows=False, key_block_pad=0, quant_dtype="e4m3",
-                dtype_scale="fp32"):
+                dtype_scale="fp32", init_num=0, local_num=0):
     """A random problem of the given layout; lengths are ragged when asked.
 
     BSND: actual lengths in [1, S] (or S when not ragged).  TND: per-sequence
@@ -295,7 +297,8 @@ def make_random(seed: int, *, layout_q="BSND", layout_k="BSND", dtype_qk="bf16",
     inputs: Dict[str, Optional[torch.Tensor]] = {}
     p = Problem(layout_q=layout_q, layout_k=layout_k, dtype_qk=qdt, dtype_w=dtype_w,
                 quant=quant, B=B, N1=N1, N2=N2, D=D, sparse_count=sparse_count,
-                sparse_mode=sparse_mode, return_value=return_value)
+                sparse_mode=sparse_mode, return_value=return_value, init_num=init_num,
+                local_num=local_num)
     # query
     if layout_q == "BSND":
         p.S1 = S1

@@ -75,6 +75,18 @@ def brute(p, inputs):
                 vis = np.ones(Sk, dtype=bool)
             tv = t_all[vis]
             sv = score[i, vis]
+            init_num = getattr(p, "init_num", 0)
+            local_num = getattr(p, "local_num", 0)
+            if init_num or local_num:
+                # sink tokens and the local window are kept whatever their
+                # score; the best of the other visible keys fill the rest
+                nv = len(tv)
+                forced = (tv < init_num) | (tv >= nv - local_num)
+                others = np.flatnonzero(~forced)
+                others = others[np.lexsort((tv[others], -sv[others]))]
+                keep = np.concatenate([np.flatnonzero(forced),
+                                       others[:max(0, min(kk, nv) - int(forced.sum()))]])
+                tv, sv = tv[keep], sv[keep]
             order = np.lexsort((tv, -sv))
             n = min(kk, len(order))
             idx[q0 + i, :n] = tv[order[:n]]

@@ -71,6 +71,8 @@ CASES = [
          dtype_scale="fp16", dtype_w="fp16"),
     dict(layout_q="BSND", layout_k="PA_BSND", sparse_mode=0, quant=True, quant_dtype="int8",
          dtype_w="fp32", block_size=16),
+    dict(layout_q="BSND", layout_k="BSND", sparse_mode=3, init_num=2, local_num=3),
+    dict(layout_q="TND", layout_k="PA_BSND", sparse_mode=0, block_size=16, init_num=4, local_num=1),
 ]
 
 
@@ -359,6 +361,46 @@ def test_int8_quantizer_round_trip():
     assert torch.all(codes.abs().to(torch.int32).amax(-1) == 127)
 
 
+def test_sink_and_local_hand_worked_example():
+    """One head, unit weight, D=1: s(t) = relu(q*k_t).  Keys 0..7 score
+    0,5,1,7,2,6,3,4 (q=1); with k=4, init_num=1, local_num=1 the sink key 0
+    (score 0) and the local key 7 (score 4) are kept whatever their score, and
+    the two best others (keys 3 and 5) fill the rest; order by score desc."""
+    q = torch.ones(1, 1, 1, 1)
+    k = torch.tensor([0.0, 5, 1, 7, 2, 6, 3, 4]).reshape(1, 8, 1, 1)
+    w = torch.ones(1, 1, 1)
+    p = synth.Problem(B=1, S1=1, S2=8, N1=1, D=1, sparse_count=4, sparse_mode=0,
+                      return_value=1, dtype_qk="bf16", dtype_w="bf16", init_num=1, local_num=1)
+    inp = dict(query=q.to(torch.bfloat16), key=k.to(torch.bfloat16), weights=w.to(torch.bfloat16))
+    o = oracle.run(p, inp)
+    np.testing.assert_array_equal(o["idx"][0], [3, 5, 7, 0])
+    np.testing.assert_array_equal(o["v64"][0], [7.0, 6.0, 4.0, 0.0])
+    p.local_num = 3                                  # keys 0, 5, 6, 7 forced: they fill k = 4
+    o = oracle.run(p, inp)
+    np.testing.assert_array_equal(o["idx"][0], [5, 7, 6, 0])
+
+
+def test_sink_and_local_keys_always_kept():
+    """Every row keeps its first init_num and last local_num visible keys,
+    the output stays ordered, and the other kept keys beat every dropped one."""
+    p, inp = small(81, layout_q="BSND", layout_k="BSND", sparse_mode=3, S1=30, S2=60,
+                   sparse_count=10, init_num=3, local_num=4)
+    o = oracle.run(p, inp, want_scores=True)
+    for r in range(p.rows):
+        nv = int(o["nvis"][r])
+        got = [int(t) for t in o["idx"][r] if t >= 0]
+        assert len(got) == min(nv, p.sparse_count)
+        forced = set(range(min(3, nv))) | set(range(max(0, nv - 4), nv))
+        assert forced <= set(got)
+        v = o["v64"][r][:len(got)]
+        assert np.all(np.diff(v) <= 0)
+        others = [t for t in got if t not in forced]
+        dropped = [t for t in range(nv) if t not in set(got)]
+        if others and dropped:
+            sc = o["scores"][r]
+            assert min(sc[t] for t in others) >= max(sc[t] for t in dropped)
+
+
 def test_quant_power_of_two_scale_equivariance():
     """Uniform positive scales c_q, c_k scale every score by c_q*c_k exactly."""
     p, inp = small(61, layout_q="TND", layout_k="TND", sparse_mode=0, quant=True, dtype_w="fp32")
@@ -402,7 +444,7 @@ def test_row_subset_matches_full_run():
 def _pin_suite(mutation):
     """Run a cross-section of the pins against a (possibly mutated) oracle."""
     failures = 0
-    for ci in (1, 3, 5, 9):
+    for ci in (1, 3, 5, 9, 14):
         p, inp = small(200 + ci, **CASES[ci])
         inp = integerize(p, inp, 200 + ci, scale_pow2=True)
         try:
@@ -416,6 +458,6 @@ def test_unmutated_oracle_passes_pin_suite():
     assert _pin_suite(0) == 0
 
 
-@pytest.mark.parametrize("mutation", [1, 2, 3, 4, 5, 6])
+@pytest.mark.parametrize("mutation", [1, 2, 3, 4, 5, 6, 7])
 def test_each_planted_mistake_is_caught(mutation):
     assert _pin_suite(mutation) > 0

@@ -88,6 +88,12 @@ typedef enum { LI_BSND = 0, LI_TND = 1, LI_PA_BSND = 2 } li_layout;
  *   max_seqlen_k   host-side upper bound on every actual key length (0 = S2 for
  *                  BSND, T2 for TND, max_blocks_per_seq*block_size for PA).  It
  *                  sizes the workspace; longer actual lengths are clamped and flagged.
+ *   init_num, local_num  sink tokens and local window (the MT lightning_indexer
+ *                  attributes of the open-sourcing issue): the first init_num and
+ *                  the last local_num visible keys of every row are always
+ *                  selected, the best other visible keys fill the remaining
+ *                  slots, all ordered by score.  0 = off; init_num + local_num
+ *                  must not exceed sparse_count.
  */
 typedef struct {
     int32_t layout_q, layout_k;
@@ -99,6 +105,7 @@ typedef struct {
     int64_t pre_tokens, next_tokens;
     int32_t return_value;
     int32_t max_seqlen_k;
+    int32_t init_num, local_num;
 } li_params;
 
 /*

@@ -54,6 +54,7 @@ class Params(ctypes.Structure):
         ("sparse_count", ctypes.c_int32), ("sparse_mode", ctypes.c_int32),
         ("pre_tokens", ctypes.c_int64), ("next_tokens", ctypes.c_int64),
         ("return_value", ctypes.c_int32), ("max_seqlen_k", ctypes.c_int32),
+        ("init_num", ctypes.c_int32), ("local_num", ctypes.c_int32),
     ]
 
 

@@ -89,6 +89,10 @@ li_status check_params(const li_params *pp, bool quant)
     if (p.return_value != 0 && p.return_value != 1)
         return fail(LI_ERR_SHAPE, "return_value must be 0 or 1");
     if (p.max_seqlen_k < 0) return fail(LI_ERR_SHAPE, "max_seqlen_k must be >= 0");
+    if (p.init_num < 0 || p.local_num < 0)
+        return fail(LI_ERR_SHAPE, "init_num and local_num must be >= 0");
+    if ((int64_t)p.init_num + p.local_num > p.sparse_count)
+        return fail(LI_ERR_SHAPE, "init_num + local_num must not exceed sparse_count");
     if (quant) {
         if (p.dtype_qk != LI_FP8_E4M3 && p.dtype_qk != LI_INT8)
             return fail(LI_ERR_DTYPE, "li_quant_indexer takes fp8 e4m3 or int8 query/key");
@@ -396,6 +400,8 @@ li_status run(const li_params *pp, bool quant, const void *query, const void *ke
     ta.kmax = (p.sparse_count + 31) & ~31;
     ta.cap = topk_cap(w.ld, p.sparse_count, ta.kmax);
     ta.standalone = 0;
+    ta.init_num = p.init_num;
+    ta.local_num = p.local_num;
     e = launch_topk(ta, s);
     if (e != cudaSuccess) return fail(LI_ERR_CUDA, "top-k launch: %s", cudaGetErrorString(e));
     ++g_launches;

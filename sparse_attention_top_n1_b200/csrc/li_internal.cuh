@@ -114,6 +114,7 @@ struct TopkArgs {
     int32_t cap;                     // row elements cached in shared memory
     int32_t kmax;                    // capacity of the selection buffers (>= k)
     int32_t standalone;
+    int32_t init_num, local_num;     // always-selected sink keys and local window
 };
 
 size_t topk_smem_bytes(int cap, int kmax);

@@ -153,9 +153,12 @@ struct TopkShared {
 // Exact for every input (ties, equal values, any range): three histogram
 // passes find the k-th key, an index-order compaction selects, a stable LSB
 // radix sort orders.  Used when the bucket path declines a row.
+// Keys j < fa and j >= fc are forced (sink tokens and local window): they
+// take part in the selection as the largest possible key and are ordered by
+// their real key (fa = 0, fc = n: none forced).
 template <int NT>
 __device__ void radix_topk(const RowSrc &src, int n, int k, int m, const TopkSmem &s,
-                           TopkShared &sh, int32_t *oidx, float *oval)
+                           TopkShared &sh, int32_t *oidx, float *oval, int fa, int fc)
 {
     constexpr int kTopkThreads = NT, kWarps = NT / 32;
     constexpr int kSortMaxRounds = 2048 / NT;       // rounds of 32 per warp for kmax <= 2048
@@ -191,8 +194,9 @@ __device__ void radix_topk(const RowSrc &src, int n, int k, int m, const TopkSme
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int j = j4 * 4 + e;
-                    const bool act = j < n && (kv[e] & pmask) == prefix;
-                    const uint32_t d = act ? (kv[e] >> shift) & dmask : 0xFFFFFFFFu;
+                    const uint32_t sk = (j < fa || j >= fc) ? 0xFFFFFFFFu : kv[e];   // selection key
+                    const bool act = j < n && (sk & pmask) == prefix;
+                    const uint32_t d = act ? (sk >> shift) & dmask : 0xFFFFFFFFu;
                     const uint32_t peers = __match_any_sync(0xffffffffu, d);
                     if (act && (peers & lanemask_lt()) == 0)
                         atomicAdd(&hist[d], (uint32_t)__popc(peers));
@@ -251,7 +255,8 @@ __device__ void radix_topk(const RowSrc &src, int n, int k, int m, const TopkSme
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int j = j4 * 4 + e;
-                    if (j < n) { ngt += kv[e] > T; neq += kv[e] == T; }
+                    const uint32_t sk = (j < fa || j >= fc) ? 0xFFFFFFFFu : kv[e];
+                    if (j < n) { ngt += sk > T; neq += sk == T; }
                 }
             }
             uint64_t packed = ((uint64_t)neq << 32) | ngt, tot;
@@ -263,7 +268,8 @@ __device__ void radix_topk(const RowSrc &src, int n, int k, int m, const TopkSme
                 for (int e = 0; e < 4; ++e) {
                     const int j = j4 * 4 + e;
                     if (j >= n) break;
-                    const bool gt = kv[e] > T, eq = kv[e] == T;
+                    const uint32_t sk = (j < fa || j >= fc) ? 0xFFFFFFFFu : kv[e];
+                    const bool gt = sk > T, eq = sk == T;
                     if (gt || (eq && eq_b < (uint32_t)need_eq)) {
                         const uint32_t pos = gt_b + (eq_b < (uint32_t)need_eq ? eq_b : (uint32_t)need_eq);
                         keyA[pos] = kv[e];
@@ -600,8 +606,11 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a)
     if (cached) src.c = s.cache;
     __syncthreads();
 
-    if (!bucket_topk(src, n, k, m, a.kmax, s, sh, oidx, oval))
-        radix_topk<kTopkThreads>(src, n, k, m, s, sh, oidx, oval);
+    // sink tokens [0, fa) and the local window [fc, n) are always selected
+    const int fa = a.init_num < n ? a.init_num : n;
+    const int fc = (n - a.local_num) > fa ? n - a.local_num : fa;
+    if (fa > 0 || fc < n || !bucket_topk(src, n, k, m, a.kmax, s, sh, oidx, oval))
+        radix_topk<kTopkThreads>(src, n, k, m, s, sh, oidx, oval, fa, fc);
 }
 
 // Number of candidate keys of a row: the visible prefix of the batch's keys
@@ -714,6 +723,9 @@ __global__ void __launch_bounds__(NT) topk_cluster_kernel(TopkArgs a)
     uint32_t *gcnt = tail + 2 * kCandLimit;
 
     const float *grow = a.scores + (int64_t)row * a.ld;
+    // sink tokens [0, fa) and the local window [fc, n) are always selected
+    const int fa = a.init_num < n ? a.init_num : n;
+    const int fc = (n - a.local_num) > fa ? n - a.local_num : fa;
     // whole row with the exact radix method, streamed from global memory (CTA 0)
     auto radix_row = [&]() {
         TopkSmem s;
@@ -726,9 +738,9 @@ __global__ void __launch_bounds__(NT) topk_cluster_kernel(TopkArgs a)
         full.g = grow;
         full.c = nullptr;
         full.n = n;
-        radix_topk<NT>(full, n, k, m, s, sh, oidx, oval);
+        radix_topk<NT>(full, n, k, m, s, sh, oidx, oval, fa, fc);
     };
-    if (n > C * NT * EPT) {             // longer than the registers hold
+    if (n > C * NT * EPT || fa > 0 || fc < n) {   // too long, or keys forced in
         if (rank == 0) radix_row();
         return;
     }

@@ -9,7 +9,11 @@ The rule (tolerance |g - o| <= atol + rtol*|o|; bf16/fp16/int8: rtol 2e-3, atol
   * every key whose oracle score exceeds s_k + tol(s_k) is selected, and every
     selected key has an oracle score >= s_k - tol(s_k), where s_k is the
     oracle's k-th value: swaps are allowed only inside the tolerance band
-    around the k-th score.
+    around the k-th score;
+  * with sink tokens / a local window, the forced keys (the first init_num and
+    last local_num visible keys) are all selected, and the band rule above
+    applies to the other keys, with s_k the oracle's k'-th best other score
+    (k' = min(k, visible) - number of forced keys).
 """
 from __future__ import annotations
 
@@ -48,16 +52,28 @@ def compare_rows(p, gpu_idx, gpu_val, orc, rows_label=None, rtol=None, atol=None
         assert len(np.unique(sel)) == m, "row %s: duplicate indices" % label
         s = scores[r]
         os_sorted = orc["v64"][r][:m]
-        s_k = os_sorted[m - 1]
-        tol_k = atol + rtol * abs(s_k)
         got_s = s[sel]
         assert np.all(np.isfinite(got_s)), "row %s: selected an invisible key" % label
-        assert np.all(got_s >= s_k - tol_k), (
-            "row %s: selected key below the k-th score band (min %.6g < %.6g)"
-            % (label, got_s.min(), s_k - tol_k))
-        must = np.nonzero(s[:nv] > s_k + tol_k)[0]
-        missing = np.setdiff1d(must, sel)
-        assert missing.size == 0, "row %s: missed keys %s" % (label, missing[:8])
+        init_num, local_num = getattr(p, "init_num", 0), getattr(p, "local_num", 0)
+        forced = np.zeros(nv, dtype=bool)
+        forced[:min(init_num, nv)] = True
+        forced[max(0, nv - local_num):] = True
+        f_idx = np.nonzero(forced)[0]
+        missing_forced = np.setdiff1d(f_idx, sel)
+        assert missing_forced.size == 0, "row %s: forced keys not kept %s" % (label, missing_forced[:8])
+        kk = m - f_idx.size                              # slots for the other keys
+        if kk > 0:
+            others = np.nonzero(~forced)[0]
+            s_oth = np.sort(s[others])[::-1]
+            s_k = s_oth[kk - 1]
+            tol_k = atol + rtol * abs(s_k)
+            sel_oth = sel[~forced[sel]]
+            assert np.all(s[sel_oth] >= s_k - tol_k), (
+                "row %s: selected key below the k-th score band (min %.6g < %.6g)"
+                % (label, s[sel_oth].min(), s_k - tol_k))
+            must = others[s[others] > s_k + tol_k]
+            missing = np.setdiff1d(must, sel)
+            assert missing.size == 0, "row %s: missed keys %s" % (label, missing[:8])
         if gpu_val is not None:
             gv = gpu_val[r][:m].astype(np.float64)
             assert np.all(np.diff(gv) <= 0), "row %s: values not non-increasing" % label

@@ -10,6 +10,7 @@
 from __future__ import annotations
 
 import ctypes
+import subprocess
 import json
 import os
 import re
@@ -38,9 +39,21 @@ def test_library_exports_every_declared_symbol():
     assert set(names) == set(li.EXPORTS)
 
 
-def test_params_struct_matches_header_size():
-    # int32 x16, int64, int32 x2, int64 x2, int32 x2 with natural alignment
-    assert ctypes.sizeof(li.Params) == 104
+def test_params_struct_matches_header_layout(tmp_path):
+    """The binding's li_params mirror has the C header's size and offsets
+    (checked by compiling a probe against include/li.h with the host C compiler)."""
+    fields = [name for name, _ in li.Params._fields_]
+    src = tmp_path / "probe.c"
+    src.write_text("#include <stdio.h>\n#include <stddef.h>\n#include \"li.h\"\n"
+                   "int main(void) {\n  printf(\"%zu\\n\", sizeof(li_params));\n" +
+                   "".join('  printf("%%zu\\n", offsetof(li_params, %s));\n' % f for f in fields) +
+                   "  return 0;\n}\n")
+    exe = tmp_path / "probe"
+    subprocess.check_call(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)])
+    out = [int(x) for x in subprocess.check_output([str(exe)]).split()]
+    assert out[0] == ctypes.sizeof(li.Params)
+    for f, off in zip(fields, out[1:]):
+        assert getattr(li.Params, f).offset == off, f
 
 
 @pytest.mark.parametrize("case", json.load(open(os.path.join(ROOT, "tests", "golden",
@@ -91,6 +104,8 @@ BAD = [
     (dict(dtype_qk="fp32"), "LI_ERR_DTYPE"),
     (dict(dtype_qk="e4m3"), "LI_ERR_DTYPE"),
     (dict(dtype_w="int8"), "LI_ERR_DTYPE"),
+    (dict(init_num=-1), "LI_ERR_SHAPE"),
+    (dict(init_num=10, local_num=7, sparse_count=16), "LI_ERR_SHAPE"),
     (dict(return_value=2), "LI_ERR_SHAPE"),
 ]
 

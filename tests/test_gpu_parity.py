@@ -80,6 +80,12 @@ CASES = {
                          block_size=32, N1=64, sparse_mode=3),
     "int8_bsnd_n5": dict(quant=True, quant_dtype="int8", dtype_scale="fp16", dtype_w="bf16",
                          N1=5, sparse_mode=0),
+    "sink_local_bsnd": dict(sparse_mode=3, init_num=4, local_num=8),
+    "sink_only_tnd": dict(layout_q="TND", layout_k="TND", sparse_mode=3, init_num=16),
+    "local_only_pa": dict(layout_k="PA_BSND", block_size=64, sparse_mode=0, local_num=32),
+    "sink_local_fill_k": dict(sparse_mode=3, sparse_count=16, init_num=6, local_num=10),
+    "sink_local_long_rows": dict(sparse_mode=0, S1=3, S2=20000, ragged=False, sparse_count=256,
+                                 init_num=5, local_num=7),
 }
 
 
@@ -93,7 +99,7 @@ def test_small_case_parity(name):
 
 @pytest.mark.parametrize("name", ["bsnd_mode3", "bsnd_fp16_d64_n32", "tnd_mode3", "pa48",
                                   "bsnd_n3_padded_heads", "quant_tnd", "quant_pa", "decode_pa",
-                                  "int8_tnd_fp16", "int8_pa_fp32"])
+                                  "int8_tnd_fp16", "int8_pa_fp32", "sink_local_bsnd"])
 def test_exact_integer_parity(name):
     """Small-integer inputs: every product and sum is exact in fp32, so the GPU
     must reproduce the oracle exactly, ties broken toward the lower index."""

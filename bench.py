@@ -50,13 +50,14 @@ WORKLOAD_DESC = {
     "quant_varlen": "quant varlen TND {2k,4k,8k,16k} N1=64 D=128 fp8 e4m3 + fp32 scales, k=2048 mode3",
     "quant_varlen_int8": "quant varlen TND {2k,4k,8k,16k} N1=64 D=128 int8 + fp16 scales/weights, k=2048 mode3",
     "quant_int8_pa": "quant int8 PA (VllmQuant README A3 example): B=24 S1=4 S2=512 N1=64 D=128 block 128, fp16 scales/weights, k=512 mode0",
+    "dsa_prefill_window": "DSA prefill with sink/local window: B=1 S1=S2=8192 N1=64 D=128 k=2048 mode3 bf16, init_num=16 local_num=512, values on",
 }
 RETURN_VALUE = {"tiny": 1, "cfg2": 1, "dsa_prefill": 1, "paged_decode": 0, "quant_varlen": 0,
-                "quant_varlen_int8": 0, "quant_int8_pa": 0}
+                "quant_varlen_int8": 0, "quant_int8_pa": 0, "dsa_prefill_window": 1}
 
 
 SEEDS = {"tiny": 0, "cfg2": 1, "dsa_prefill": 2, "paged_decode": 3, "quant_varlen": 4,
-         "quant_int8_pa": 5, "quant_varlen_int8": 6}
+         "quant_int8_pa": 5, "quant_varlen_int8": 6, "dsa_prefill_window": 7}
 
 
 def make_workload(name, rank=0):

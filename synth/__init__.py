@@ -216,6 +216,17 @@ def make_quant_varlen(seed: int = 4, lens=(2048, 4096, 8192, 16384), return_valu
                    act_q=cum.clone(), act_k=cum.clone())
 
 
+def make_dsa_prefill_window(seed: int = 7, return_value: int = 1, init_num: int = 16,
+                            local_num: int = 512):
+    """dsa_prefill with sink tokens and a local window (values not from the
+    pages, which name the attributes only): the first 16 and the last 512
+    visible keys of every row are always selected."""
+    p, inp = make_dsa_prefill(seed=seed, return_value=return_value)
+    p.init_num = init_num
+    p.local_num = local_num
+    return p, inp
+
+
 def make_quant_varlen_int8(seed: int = 6, return_value: int = 0):
     """quant_varlen with int8 q/k, fp16 scales and fp16 weights."""
     return make_quant_varlen(seed=seed, return_value=return_value, qdtype="int8",
@@ -258,6 +269,7 @@ WORKLOADS = {
     "quant_varlen": make_quant_varlen,
     "quant_varlen_int8": make_quant_varlen_int8,
     "quant_int8_pa": make_quant_int8_pa,
+    "dsa_prefill_window": make_dsa_prefill_window,
 }
 
 

@@ -120,6 +120,13 @@ def test_exact_integer_parity(name):
     np.testing.assert_array_equal(gv, o["val"])
 
 
+def test_dsa_prefill_window_workload_sampled():
+    p, inp = synth.make_dsa_prefill_window()
+    gi, gv, flags = run_gpu(p, inp)
+    assert flags == 0
+    check_against_oracle(p, inp, gi, gv, rows=sample_rows(p, n_random=48, edge=16))
+
+
 def test_quant_int8_readme_example_full():
     """The VllmQuantLightningIndexer README's A3 call: int8 q/k over the full
     int8 range (|q.k| up to 2^21), fp16 scales and weights, PA keys."""

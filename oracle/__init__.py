@@ -43,6 +43,7 @@ class OrProblem(ctypes.Structure):
         ("sparse_count", ctypes.c_int32), ("sparse_mode", ctypes.c_int32),
         ("return_value", ctypes.c_int32), ("mutation", ctypes.c_int32),
         ("init_num", ctypes.c_int32), ("local_num", ctypes.c_int32),
+        ("cmp_ratio", ctypes.c_int32), ("cmp_residual_k", ctypes.c_void_p),
     ]
 
 
@@ -94,7 +95,8 @@ def _ptr(a):
     return None if a is None else a.ctypes.data
 
 
-def make_problem(p, mutation: int = 0) -> OrProblem:
+def make_problem(p, mutation: int = 0, cmp_res=None) -> OrProblem:
+    """cmp_res: int32 numpy array [B] of residual original tokens (kept alive by the caller)."""
     return OrProblem(
         layout_q=LAYOUT[p.layout_q], layout_k=LAYOUT[p.layout_k],
         dtype_qk=DT[p.dtype_qk], dtype_w=DT[p.dtype_w], dtype_scale=DT[p.dtype_scale],
@@ -103,7 +105,9 @@ def make_problem(p, mutation: int = 0) -> OrProblem:
         max_blocks_per_seq=p.max_blocks_per_seq, key_block_stride=p.key_block_stride,
         sparse_count=p.sparse_count, sparse_mode=p.sparse_mode,
         return_value=p.return_value, mutation=mutation,
-        init_num=getattr(p, "init_num", 0), local_num=getattr(p, "local_num", 0))
+        init_num=getattr(p, "init_num", 0), local_num=getattr(p, "local_num", 0),
+        cmp_ratio=getattr(p, "cmp_ratio", 1),
+        cmp_residual_k=None if cmp_res is None else cmp_res.ctypes.data)
 
 
 def max_key_len(p, inputs) -> int:
@@ -127,7 +131,9 @@ def run(p, inputs, rows: Optional[Sequence[int]] = None, want_scores: bool = Fal
     asked, ``scores`` [n, ld] float64 (NaN where a key is not visible).
     """
     L = lib()
-    prob = make_problem(p, mutation)
+    cmp_res = inputs.get("cmp_residual_k")
+    cmp_res = None if cmp_res is None else np.ascontiguousarray(cmp_res.numpy().astype(np.int32))
+    prob = make_problem(p, mutation, cmp_res)
     k = p.sparse_count
     if rows is None:
         rows_arr = None

@@ -36,7 +36,13 @@
  *   - the deterministic Top-k breaks ties toward the lower key index;
  *   - indices are positions inside the batch's own key sequence;
  *   - TND actual lengths are prefix sums (no leading 0), BSND/PA are counts;
- *   - BSND rows with i >= actual query length are pure padding.
+ *   - BSND rows with i >= actual query length are pure padding;
+ *   - compressed keys (CANN LightningIndexerV2 guide: cmp_ratio, with
+ *     cmp_residual_k < cmp_ratio under mask_mode 3): compressed key t stands
+ *     for the cmp_ratio original tokens [t*r, (t+1)*r); the batch's original
+ *     key length is Sk*r + residual; under right-down causal masking t is
+ *     visible once its last original token (t+1)*r - 1 is, i.e. when
+ *     (t+1)*r - 1 <= i + Sk*r + residual - Sq.  Indices count compressed keys.
  *
  * Planted mistakes: the field `mutation` (0 in every real use) lets the tests
  * inject one deliberate error at a time into this oracle, to show that each
@@ -63,6 +69,8 @@ typedef struct {
     int32_t sparse_count, sparse_mode, return_value;
     int32_t mutation;              /* 0 = the real oracle; >0 plants one mistake */
     int32_t init_num, local_num;   /* forced sink tokens / local window (0 = none) */
+    int32_t cmp_ratio;             /* original tokens per key (0 or 1 = none) */
+    const int32_t *cmp_residual_k; /* [B] leftover original tokens (mode 3, cmp_ratio > 1) */
 } or_problem;
 
 /* ---- decoders, from the format definitions ------------------------------ */
@@ -120,7 +128,7 @@ double li_oracle_decode(const void *base, int64_t i, int dtype) { return load(ba
 
 /* ---- sequence bookkeeping (mindspore page, "actual_seq_lengths_*") -------- */
 
-typedef struct { int64_t q_off, k_off; int64_t Sq, Sk; } seq_info;
+typedef struct { int64_t q_off, k_off; int64_t Sq, Sk; int64_t res; } seq_info;
 
 static seq_info seq_of(const or_problem *p, const int32_t *act_q, const int32_t *act_k, int b)
 {
@@ -142,6 +150,7 @@ static seq_info seq_of(const or_problem *p, const int32_t *act_q, const int32_t 
         s.k_off = 0;
         s.Sk = act_k[b];
     }
+    s.res = (p->cmp_ratio > 1 && p->sparse_mode == 3 && p->cmp_residual_k) ? p->cmp_residual_k[b] : 0;
     return s;
 }
 
@@ -178,9 +187,12 @@ static int visible(const or_problem *p, seq_info s, int64_t i, int64_t t)
         return 0;
     if (p->sparse_mode == 0)
         return 1;
+    const int64_t r = p->cmp_ratio > 1 ? p->cmp_ratio : 1;
+    const int64_t last_tok = (t + 1) * r - 1;            /* last original token of key t */
+    const int64_t diag = i + s.Sk * r + s.res - s.Sq;    /* right-down causal, original tokens */
     if (p->mutation == 4)                      /* planted: off-by-one diagonal */
-        return t < i + s.Sk - s.Sq;
-    return t <= i + s.Sk - s.Sq;
+        return last_tok < diag;
+    return last_tok <= diag;
 }
 
 typedef struct { double s; int64_t t; } cand;
@@ -367,4 +379,4 @@ int li_oracle_rows(const or_problem *p, const void *query, const void *key, cons
     return bad ? -1 : 0;
 }
 
-int li_oracle_abi_version(void) { return 2; }
+int li_oracle_abi_version(void) { return 3; }

@@ -77,6 +77,7 @@ class Problem:
     max_seqlen_k: int = 0           # host-side bound on any key length (0 = derive)
     init_num: int = 0               # sink tokens always selected (first visible keys)
     local_num: int = 0              # local window always selected (last visible keys)
+    cmp_ratio: int = 1              # original tokens per (compressed) key
 
     @property
     def rows(self) -> int:
@@ -227,6 +228,23 @@ def make_dsa_prefill_window(seed: int = 7, return_value: int = 1, init_num: int 
     return p, inp
 
 
+def make_v2_compressed(seed: int = 8, return_value: int = 1):
+    """The CANN LightningIndexerV2 guide's call example (section 调用示例):
+    B=2, S1=64, S2=130 original key tokens compressed by cmp_ratio=4 into
+    32 keys with 2 residual tokens per batch, N1=16, D=128, topk=32,
+    mask_mode 3, fp16 q/k, fp32 weights, all N(0,1)."""
+    B, S1, S2, r, N1, D = 2, 64, 130, 4, 16, 128
+    g = _gen(seed)
+    q = _normal(g, (B, S1, N1, D), "fp16")
+    k = _normal(g, (B, S2 // r, 1, D), "fp16")
+    w = torch.randn(B, S1, N1, generator=g, dtype=torch.float32)
+    p = Problem(layout_q="BSND", layout_k="BSND", dtype_qk="fp16", dtype_w="fp32",
+                B=B, S1=S1, S2=S2 // r, N1=N1, N2=1, D=D, sparse_count=32, sparse_mode=3,
+                return_value=return_value, cmp_ratio=r)
+    return p, dict(query=q, key=k, weights=w,
+                   cmp_residual_k=torch.full((B,), S2 % r, dtype=torch.int32))
+
+
 def make_quant_varlen_int8(seed: int = 6, return_value: int = 0):
     """quant_varlen with int8 q/k, fp16 scales and fp16 weights."""
     return make_quant_varlen(seed=seed, return_value=return_value, qdtype="int8",
@@ -270,6 +288,7 @@ WORKLOADS = {
     "quant_varlen_int8": make_quant_varlen_int8,
     "quant_int8_pa": make_quant_int8_pa,
     "dsa_prefill_window": make_dsa_prefill_window,
+    "v2_compressed": make_v2_compressed,
 }
 
 
@@ -281,7 +300,7 @@ def make_random(seed: int, *, layout_q="BSND", layout_k="BSND", dtype_qk="bf16",
                 dtype_w="bf16", B=2, S1=40, S2=300, N1=8, D=128, sparse_count=64,
                 sparse_mode=3, return_value=1, ragged=True, block_size=64,
                 quant=False, empty_rows=False, key_block_pad=0, quant_dtype="e4m3",
-                dtype_scale="fp32", init_num=0, local_num=0):
+                dtype_scale="fp32", init_num=0, local_num=0, cmp_ratio=1):
     """A random problem of the given layout; lengths are ragged when asked.
 
     BSND: actual lengths in [1, S] (or S when not ragged).  TND: per-sequence
@@ -310,7 +329,10 @@ def make_random(seed: int, *, layout_q="BSND", layout_k="BSND", dtype_qk="bf16",
     p = Problem(layout_q=layout_q, layout_k=layout_k, dtype_qk=qdt, dtype_w=dtype_w,
                 quant=quant, B=B, N1=N1, N2=N2, D=D, sparse_count=sparse_count,
                 sparse_mode=sparse_mode, return_value=return_value, init_num=init_num,
-                local_num=local_num)
+                local_num=local_num, cmp_ratio=cmp_ratio)
+    if cmp_ratio > 1 and sparse_mode == 3:
+        # leftover original tokens per batch, each below cmp_ratio
+        inputs["cmp_residual_k"] = torch.randint(0, cmp_ratio, (B,), generator=g).to(torch.int32)
     # query
     if layout_q == "BSND":
         p.S1 = S1

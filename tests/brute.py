@@ -68,9 +68,14 @@ def brute(p, inputs):
             logits = logits * qs[q0:q0 + Sq][:, :, None] * KS[None, None, :]
         score = (np.maximum(logits, 0.0) * W[:, :, None]).sum(axis=1)   # [Sq, Sk]
         t_all = np.arange(Sk)
+        r = max(1, getattr(p, "cmp_ratio", 1))
+        res = int(inputs["cmp_residual_k"][b]) if (r > 1 and p.sparse_mode == 3) else 0
         for i in range(Sq):
             if p.sparse_mode == 3:
-                vis = t_all <= i + Sk - Sq
+                # compressed key t covers original tokens [t*r, (t+1)*r); the
+                # original keys number Sk*r + res; count the visible ones
+                nvis = max(0, min(Sk, (i + 1 - Sq + Sk * r + res) // r))
+                vis = t_all < nvis
             else:
                 vis = np.ones(Sk, dtype=bool)
             tv = t_all[vis]

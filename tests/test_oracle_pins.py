@@ -73,6 +73,8 @@ CASES = [
          dtype_w="fp32", block_size=16),
     dict(layout_q="BSND", layout_k="BSND", sparse_mode=3, init_num=2, local_num=3),
     dict(layout_q="TND", layout_k="PA_BSND", sparse_mode=0, block_size=16, init_num=4, local_num=1),
+    dict(layout_q="BSND", layout_k="BSND", sparse_mode=3, cmp_ratio=4),
+    dict(layout_q="TND", layout_k="PA_BSND", sparse_mode=3, block_size=16, cmp_ratio=2),
 ]
 
 
@@ -361,6 +363,31 @@ def test_int8_quantizer_round_trip():
     assert torch.all(codes.abs().to(torch.int32).amax(-1) == 127)
 
 
+def test_v2_compressed_example_visible_counts():
+    """The CANN V2 guide's example: S2 = 130 original tokens, cmp_ratio = 4,
+    so 32 compressed keys and 2 residual tokens; with S1 = 64 right-down
+    causal queries, query i sees the compressed keys whose 4 tokens all lie at
+    or before original position i + 130 - 64, i.e. floor((i + 67) / 4) of
+    them (16 for the first query, all 32 for the last)."""
+    p, inp = synth.make_v2_compressed()
+    o = oracle.run(p, inp)
+    expect = np.array([min(32, (i + 67) // 4) for i in range(64)] * 2)
+    np.testing.assert_array_equal(o["nvis"], expect)
+    assert expect[0] == 16 and expect[63] == 32
+    # every row keeps min(32, visible) keys, all of them visible
+    for r in range(p.rows):
+        got = o["idx"][r]
+        assert np.all(got[:min(32, expect[r])] < expect[r]) and np.all(got[expect[r]:] == -1)
+
+
+def test_cmp_ratio_one_is_the_plain_mask():
+    p, inp = small(91, layout_q="BSND", layout_k="BSND", sparse_mode=3)
+    o = oracle.run(p, inp)
+    p2 = synth.Problem(**{**p.__dict__, "cmp_ratio": 1})
+    o2 = oracle.run(p2, dict(inp, cmp_residual_k=torch.zeros(p.B, dtype=torch.int32)))
+    np.testing.assert_array_equal(o["idx"], o2["idx"])
+
+
 def test_sink_and_local_hand_worked_example():
     """One head, unit weight, D=1: s(t) = relu(q*k_t).  Keys 0..7 score
     0,5,1,7,2,6,3,4 (q=1); with k=4, init_num=1, local_num=1 the sink key 0
@@ -444,7 +471,7 @@ def test_row_subset_matches_full_run():
 def _pin_suite(mutation):
     """Run a cross-section of the pins against a (possibly mutated) oracle."""
     failures = 0
-    for ci in (1, 3, 5, 9, 14):
+    for ci in (1, 3, 5, 9, 14, 16):
         p, inp = small(200 + ci, **CASES[ci])
         inp = integerize(p, inp, 200 + ci, scale_pow2=True)
         try:

@@ -94,6 +94,17 @@ typedef enum { LI_BSND = 0, LI_TND = 1, LI_PA_BSND = 2 } li_layout;
  *                  selected, the best other visible keys fill the remaining
  *                  slots, all ordered by score.  0 = off; init_num + local_num
  *                  must not exceed sparse_count.
+ *   cmp_ratio      compressed keys (CANN LightningIndexerV2 guide): every key
+ *                  stands for cmp_ratio original tokens; 0 or 1 = none; a power
+ *                  of two up to 128.  Indices count compressed keys.
+ *   cmp_residual_k device int32 [B]: original key tokens left over after the
+ *                  last whole compressed key, each < cmp_ratio.  Required when
+ *                  cmp_ratio > 1 and sparse_mode == 3 (then a key is visible once
+ *                  all of its original tokens are: key t is visible to query i iff
+ *                  (t+1)*cmp_ratio - 1 <= i + Sk*cmp_ratio + residual - Sq);
+ *                  ignored otherwise.  A residual outside [0, cmp_ratio) is
+ *                  clamped and flagged with LI_DEV_BAD_KLEN.
+ *   reserved       must be 0
  */
 typedef struct {
     int32_t layout_q, layout_k;
@@ -106,6 +117,9 @@ typedef struct {
     int32_t return_value;
     int32_t max_seqlen_k;
     int32_t init_num, local_num;
+    int32_t cmp_ratio;
+    int32_t reserved;
+    const int32_t *cmp_residual_k;
 } li_params;
 
 /*

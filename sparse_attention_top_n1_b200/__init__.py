@@ -55,6 +55,8 @@ class Params(ctypes.Structure):
         ("pre_tokens", ctypes.c_int64), ("next_tokens", ctypes.c_int64),
         ("return_value", ctypes.c_int32), ("max_seqlen_k", ctypes.c_int32),
         ("init_num", ctypes.c_int32), ("local_num", ctypes.c_int32),
+        ("cmp_ratio", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("cmp_residual_k", ctypes.c_void_p),
     ]
 
 
@@ -225,14 +227,17 @@ def alloc_workspace(params: Params, device="cuda"):
 
 
 def indexer(params: Params, query, key, weights, *, act_seq_q=None, act_seq_k=None,
-            block_table=None, q_scale=None, k_scale=None, workspace=None, out=None,
-            stream=None):
+            block_table=None, q_scale=None, k_scale=None, cmp_residual_k=None, workspace=None,
+            out=None, stream=None):
     """Run li_indexer / li_quant_indexer, allocating outputs (and workspace).
 
-    Returns (sparse_indices, sparse_values); sparse_values is an empty (0,)
-    tensor when return_value is 0, as the CANN guide's output rule says.
+    cmp_residual_k (int32 [B] on the device) is stored into params before the
+    call.  Returns (sparse_indices, sparse_values); sparse_values is an empty
+    (0,) tensor when return_value is 0, as the CANN guide's output rule says.
     """
     import torch
+    if cmp_residual_k is not None:
+        params.cmp_residual_k = _ptr(cmp_residual_k)
     shape = li_output_shape(params)
     dev = query.device
     if out is None:

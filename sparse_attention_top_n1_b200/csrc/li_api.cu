@@ -93,6 +93,9 @@ li_status check_params(const li_params *pp, bool quant)
         return fail(LI_ERR_SHAPE, "init_num and local_num must be >= 0");
     if ((int64_t)p.init_num + p.local_num > p.sparse_count)
         return fail(LI_ERR_SHAPE, "init_num + local_num must not exceed sparse_count");
+    if (p.cmp_ratio < 0 || p.cmp_ratio > 128 || (p.cmp_ratio & (p.cmp_ratio - 1)))
+        return fail(LI_ERR_SHAPE, "cmp_ratio must be 0, 1 or a power of two up to 128");
+    if (p.reserved != 0) return fail(LI_ERR_SHAPE, "reserved must be 0");
     if (quant) {
         if (p.dtype_qk != LI_FP8_E4M3 && p.dtype_qk != LI_INT8)
             return fail(LI_ERR_DTYPE, "li_quant_indexer takes fp8 e4m3 or int8 query/key");
@@ -242,6 +245,10 @@ li_status run(const li_params *pp, bool quant, const void *query, const void *ke
     if ((p.layout_k == LI_TND || p.layout_k == LI_PA_BSND) && !act_k)
         return fail(LI_ERR_NULL, "TND/PA key needs actual_seq_lengths_key");
     if (p.layout_k == LI_PA_BSND && !block_table) return fail(LI_ERR_NULL, "PA needs block_table");
+    int cmp_shift = 0;
+    while ((1 << cmp_shift) < p.cmp_ratio) ++cmp_shift;
+    if (cmp_shift > 0 && p.sparse_mode == 3 && !p.cmp_residual_k)
+        return fail(LI_ERR_NULL, "cmp_ratio > 1 with sparse_mode 3 needs cmp_residual_k");
     if (!aligned(query, 16) || !aligned(key, 16))
         return fail(LI_ERR_SHAPE, "query and key must be 16-byte aligned");
     if (!aligned(weights, 4) || !aligned(out_idx, 4) || (out_val && !aligned(out_val, 4)))
@@ -343,6 +350,8 @@ li_status run(const li_params *pp, bool quant, const void *query, const void *ke
     pa.max_blocks = w.max_blocks;
     pa.ld = w.ld;
     pa.pa_capacity = (int64_t)p.max_blocks_per_seq * p.block_size;
+    pa.cmp_res = cmp_shift > 0 && p.sparse_mode == 3 ? p.cmp_residual_k : nullptr;
+    pa.cmp_shift = cmp_shift;
     if (!prof_mark(0, s)) return fail(LI_ERR_CUDA, "recording profile event 0 failed");
     cudaError_t e = launch_plan(pa, s);
     if (e != cudaSuccess) return fail(LI_ERR_CUDA, "scheduler launch: %s", cudaGetErrorString(e));
@@ -377,6 +386,7 @@ li_status run(const li_params *pp, bool quant, const void *query, const void *ke
     const int kind = !quant ? kKindF16 : (p.dtype_qk == LI_INT8 ? kKindI8 : kKindE4M3);
     const uint32_t fmt = kind == kKindF16 ? (p.dtype_qk == LI_BF16 ? 1u : 0u) : (kind == kKindI8 ? 1u : 0u);
     sa.idesc_base = make_idesc(fmt, fmt, 128, 0, kind == kKindI8 ? 2u : 1u);
+    sa.cmp_shift = cmp_shift;
     sa.dtype_scale = p.dtype_scale;
     sa.timeout_ns = kDefaultTimeoutNs;
     e = launch_score(sa, t, qmap, kmap, kind, sms, s);
@@ -402,6 +412,7 @@ li_status run(const li_params *pp, bool quant, const void *query, const void *ke
     ta.standalone = 0;
     ta.init_num = p.init_num;
     ta.local_num = p.local_num;
+    ta.cmp_shift = cmp_shift;
     e = launch_topk(ta, s);
     if (e != cudaSuccess) return fail(LI_ERR_CUDA, "top-k launch: %s", cudaGetErrorString(e));
     ++g_launches;

@@ -32,8 +32,20 @@ struct BatchInfo {
     int32_t blk_off;   // first query block of this batch
     int32_t row0;      // output row of i = 0
     int32_t nblk;      // query blocks of this batch
-    int32_t pad;
+    int32_t res;       // residual original key tokens (compressed keys, mode 3)
 };
+
+// Keys visible to query i under right-down causal masking (CANN
+// LightningIndexerV2 guide, sparse_mode 3, with cmp_ratio = 2^shift): each
+// key stands for 2^shift original tokens, the batch has Sk * 2^shift + res
+// original key tokens, and a key is visible once its last original token is
+// at or before position i + that length - Sq.  shift = res = 0: t <= i + Sk - Sq.
+__host__ __device__ __forceinline__ int32_t causal_visible(int64_t i, int32_t Sq, int32_t Sk,
+                                                           int32_t res, int32_t shift)
+{
+    const int64_t v = (i + 1 - Sq + ((int64_t)Sk << shift) + res) >> shift;   // floor
+    return v < 0 ? 0 : (v > Sk ? Sk : (int32_t)v);
+}
 
 // One query block: up to nq consecutive queries of one batch.
 struct BlockInfo {
@@ -80,6 +92,8 @@ struct PlanArgs {
     int64_t pa_capacity;   // max_blocks_per_seq * block_size
     int4 *cta_start;       // per score CTA: (block, tile, block's unit_start, block's ntiles)
     int32_t grid;          // score CTAs
+    const int32_t *cmp_res;  // [B] residual original key tokens (NULL: none)
+    int32_t cmp_shift;       // log2(cmp_ratio)
 };
 
 struct ScoreArgs {
@@ -99,6 +113,7 @@ struct ScoreArgs {
     int32_t q_box_rows;         // rows per Q TMA box: n1p*nq (packed) or N1 (per query)
     int32_t q_single, k_single; // one copy covers both 128-byte chunks (3-D / 4-D maps)
     uint32_t idesc_base;        // instruction descriptor without N
+    int32_t cmp_shift;          // log2(cmp_ratio): compressed keys under mode 3
     int64_t timeout_ns;
 };
 
@@ -115,6 +130,7 @@ struct TopkArgs {
     int32_t kmax;                    // capacity of the selection buffers (>= k)
     int32_t standalone;
     int32_t init_num, local_num;     // always-selected sink keys and local window
+    int32_t cmp_shift;               // log2(cmp_ratio): compressed keys under mode 3
 };
 
 size_t topk_smem_bytes(int cap, int kmax);

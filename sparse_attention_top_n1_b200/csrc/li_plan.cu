@@ -60,15 +60,14 @@ __device__ int32_t block_inclusive_scan(int32_t &v, int32_t *tmp)
     return total;
 }
 
-constexpr int kSmemBatches = 1024;      // batches mirrored in shared memory
+constexpr int kSmemBatches = 768;       // batches mirrored in shared memory
 constexpr int kSmemBlocks = 8192;       // query blocks whose first unit is mirrored
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a)
 {
     __shared__ int32_t s_tmp[kPlanThreads / 32];
     __shared__ int32_t s_flags;
-    __shared__ int32_t s_blk_off[kSmemBatches];
-    __shared__ int2 s_len[kSmemBatches];          // (Sq, Sk)
+    __shared__ int4 s_bat[kSmemBatches];          // (blk_off, Sq, Sk, res)
     __shared__ int32_t s_ustart[kSmemBlocks];     // unit_start of block g
     const bool in_smem = a.B <= kSmemBatches;
     const int tid = threadIdx.x;
@@ -124,6 +123,11 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a)
             bi.row0 = (int32_t)q_off;
             nblk = (int32_t)((Sq + a.nq - 1) / a.nq);
             bi.nblk = nblk;
+            if (a.cmp_res && a.mode == 3) {           // residual tokens: below cmp_ratio
+                const int32_t r = a.cmp_res[b], rmax = (1 << a.cmp_shift) - 1;
+                bi.res = r < 0 ? 0 : (r > rmax ? rmax : r);
+                if (bi.res != r) flags |= LI_DEV_BAD_KLEN;
+            }
         }
         if (flags) atomicOr(&s_flags, flags);
         int32_t incl = nblk;
@@ -132,8 +136,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a)
             bi.blk_off = carry + incl - nblk;
             a.batches[b] = bi;
             if (in_smem) {
-                s_blk_off[b] = bi.blk_off;
-                s_len[b] = make_int2(bi.Sq, bi.Sk);
+                s_bat[b] = make_int4(bi.blk_off, bi.Sq, bi.Sk, bi.res);
             }
         }
         carry += tot;
@@ -157,26 +160,29 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a)
             int lo = 0, hi = a.B - 1;                  // last batch with blk_off <= g
             while (lo < hi) {
                 const int mid = (lo + hi + 1) >> 1;
-                const int off = in_smem ? s_blk_off[mid] : a.batches[mid].blk_off;
+                const int off = in_smem ? s_bat[mid].x : a.batches[mid].blk_off;
                 if (off <= g) lo = mid; else hi = mid - 1;
             }
-            int32_t blk_off, Sq, Sk;
+            int32_t blk_off, Sq, Sk, res;
             if (in_smem) {
-                blk_off = s_blk_off[lo];
-                Sq = s_len[lo].x;
-                Sk = s_len[lo].y;
+                const int4 sb = s_bat[lo];
+                blk_off = sb.x;
+                Sq = sb.y;
+                Sk = sb.z;
+                res = sb.w;
             } else {
                 const BatchInfo bi = a.batches[lo];
                 blk_off = bi.blk_off;
                 Sq = bi.Sq;
                 Sk = bi.Sk;
+                res = bi.res;
             }
             const int32_t i0 = (g - blk_off) * a.nq;
             int32_t i_last = i0 + a.nq;
             if (i_last > Sq) i_last = Sq;
             i_last -= 1;
             int64_t nvis = Sk;
-            if (a.mode == 3) nvis = clamp64((int64_t)i_last + 1 + Sk - Sq, 0, Sk);
+            if (a.mode == 3) nvis = causal_visible(i_last, Sq, Sk, res, a.cmp_shift);
             ntiles = (int32_t)((nvis + kTileKeys - 1) / kTileKeys);
             blk.b = lo;
             blk.i0 = i0;

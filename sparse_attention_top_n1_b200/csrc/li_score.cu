@@ -533,7 +533,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             BlockInfo blk{};
             BatchInfo bi{};
             float *row_ptr = nullptr;              // score row of this half's first query
-            int lim0 = 0, nq_valid = 0;            // visible limit of that query; valid queries
+            int64_t lim0 = 0;                      // visible keys of query q: (lim0 + q) >> cmp_shift
+            int nq_valid = 0;                      // valid queries of this warp
             for (; w.valid(); w.next()) {
                 if (w.qb != prev_qb) {
                     blk = a.blocks[w.qb];
@@ -546,7 +547,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                     nchunks = (mine * N1P + 31) / 32;
                     const int i_first = blk.i0 + half * QPW;
                     row_ptr = a.scores + (int64_t)(bi.row0 + i_first) * a.ld;
-                    lim0 = a.mode == 3 ? i_first + 1 + bi.Sk - bi.Sq : bi.Sk;
+                    // right-down causal over compressed keys (see causal_visible);
+                    // mode 0 sees all Sk keys
+                    lim0 = a.mode == 3
+                               ? (int64_t)i_first + 1 - bi.Sq + ((int64_t)bi.Sk << a.cmp_shift) + bi.res
+                               : ((int64_t)bi.Sk << a.cmp_shift);
                     __syncwarp();
                     for (int j = lane; j < 128; j += 32) {
                         const int col = half * 128 + j;
@@ -613,8 +618,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 #pragma unroll
                 for (int q = 0; q < QPW; ++q) {
                     if (q < nq_valid) {
-                        int nv = lim0 + q;
-                        nv = nv < 0 ? 0 : (nv < bi.Sk ? nv : bi.Sk);
+                        const int64_t v = (lim0 + q) >> a.cmp_shift;
+                        const int nv = v < 0 ? 0 : (v < bi.Sk ? (int)v : bi.Sk);
                         if (t < nv) {
                             float s = 0.f;
 #pragma unroll

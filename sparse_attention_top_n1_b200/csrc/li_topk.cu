@@ -538,14 +538,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a)
             i = row - a.batches[b].q_off;
         }
         const BatchInfo bi = a.batches[b];
-        if (i >= 0 && i < bi.Sq) {
-            int nv = bi.Sk;
-            if (a.mode == 3) {
-                int lim = i + 1 + bi.Sk - bi.Sq;
-                nv = lim < 0 ? 0 : (lim < bi.Sk ? lim : bi.Sk);
-            }
-            n = nv;
-        }
+        if (i >= 0 && i < bi.Sq)
+            n = a.mode == 3 ? causal_visible(i, bi.Sq, bi.Sk, bi.res, a.cmp_shift) : bi.Sk;
     }
     int32_t *oidx = a.out_idx + (int64_t)row * k;
     float *oval = a.out_val ? a.out_val + (int64_t)row * k : nullptr;
@@ -637,8 +631,7 @@ __device__ __forceinline__ int row_length(const TopkArgs &a, int row)
     const BatchInfo bi = a.batches[b];
     if (i < 0 || i >= bi.Sq) return 0;
     if (a.mode != 3) return bi.Sk;
-    const int lim = i + 1 + bi.Sk - bi.Sq;
-    return lim < 0 ? 0 : (lim < bi.Sk ? lim : bi.Sk);
+    return causal_visible(i, bi.Sq, bi.Sk, bi.res, a.cmp_shift);
 }
 
 template <int NT>

@@ -105,6 +105,8 @@ BAD = [
     (dict(dtype_qk="e4m3"), "LI_ERR_DTYPE"),
     (dict(dtype_w="int8"), "LI_ERR_DTYPE"),
     (dict(init_num=-1), "LI_ERR_SHAPE"),
+    (dict(cmp_ratio=3), "LI_ERR_SHAPE"),
+    (dict(cmp_ratio=256), "LI_ERR_SHAPE"),
     (dict(init_num=10, local_num=7, sparse_count=16), "LI_ERR_SHAPE"),
     (dict(return_value=2), "LI_ERR_SHAPE"),
 ]

@@ -30,7 +30,8 @@ def run_gpu(p, inputs):
     ws = li.alloc_workspace(pr)
     idx, val = li.indexer(pr, d["query"], d["key"], d["weights"], act_seq_q=d.get("act_q"),
                           act_seq_k=d.get("act_k"), block_table=d.get("block_table"),
-                          q_scale=d.get("q_scale"), k_scale=d.get("k_scale"), workspace=ws)
+                          q_scale=d.get("q_scale"), k_scale=d.get("k_scale"),
+                          cmp_residual_k=d.get("cmp_residual_k"), workspace=ws)
     assert li.li_last_launch_count() == 3
     flags = li.li_read_device_status(ws)
     torch.cuda.synchronize()
@@ -86,6 +87,11 @@ CASES = {
     "sink_local_fill_k": dict(sparse_mode=3, sparse_count=16, init_num=6, local_num=10),
     "sink_local_long_rows": dict(sparse_mode=0, S1=3, S2=20000, ragged=False, sparse_count=256,
                                  init_num=5, local_num=7),
+    "cmp4_bsnd": dict(sparse_mode=3, cmp_ratio=4),
+    "cmp2_tnd_q_pa_k": dict(layout_q="TND", layout_k="PA_BSND", block_size=32, sparse_mode=3,
+                            cmp_ratio=2),
+    "cmp128_bsnd_n64": dict(sparse_mode=3, cmp_ratio=128, N1=64, S1=40, S2=300),
+    "cmp8_mode0": dict(sparse_mode=0, cmp_ratio=8),
 }
 
 
@@ -99,7 +105,7 @@ def test_small_case_parity(name):
 
 @pytest.mark.parametrize("name", ["bsnd_mode3", "bsnd_fp16_d64_n32", "tnd_mode3", "pa48",
                                   "bsnd_n3_padded_heads", "quant_tnd", "quant_pa", "decode_pa",
-                                  "int8_tnd_fp16", "int8_pa_fp32", "sink_local_bsnd"])
+                                  "int8_tnd_fp16", "int8_pa_fp32", "sink_local_bsnd", "cmp4_bsnd"])
 def test_exact_integer_parity(name):
     """Small-integer inputs: every product and sum is exact in fp32, so the GPU
     must reproduce the oracle exactly, ties broken toward the lower index."""
@@ -118,6 +124,15 @@ def test_exact_integer_parity(name):
     o = oracle.run(p, inp)
     np.testing.assert_array_equal(gi, o["idx"])
     np.testing.assert_array_equal(gv, o["val"])
+
+
+def test_v2_compressed_example_full():
+    """The CANN V2 guide's call example: 130 original key tokens compressed
+    4:1 into 32 keys with 2 residual tokens, right-down causal over them."""
+    p, inp = synth.make_v2_compressed()
+    gi, gv, flags = run_gpu(p, inp)
+    assert flags == 0
+    check_against_oracle(p, inp, gi, gv)
 
 
 def test_dsa_prefill_window_workload_sampled():
@@ -235,6 +250,15 @@ def test_topk_stage_exact(ld, k, kind):
 
 
 # ------------------------------------------------------------------ device status word
+
+def test_device_flag_bad_cmp_residual():
+    """A residual outside [0, cmp_ratio) is clamped and flagged, not trusted."""
+    p, inp = small(9, sparse_mode=3, cmp_ratio=4)
+    inp = dict(inp)
+    inp["cmp_residual_k"] = torch.tensor([5, 1], dtype=torch.int32)
+    _, _, flags = run_gpu(p, inp)
+    assert flags & li.DEV_BAD_KLEN
+
 
 def test_device_flags_bad_lengths_and_blocks():
     p, inp = small(3, layout_k="PA_BSND", block_size=64, sparse_mode=3)

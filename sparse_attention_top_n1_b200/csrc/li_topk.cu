@@ -681,8 +681,10 @@ constexpr int kCBuckets = 2048;      // 52 KB per CTA: the 512 CTAs of 64 long r
 // slice keys 4*(t + g*NT) .. +3).  Selected keys travel as one 64-bit word,
 // (order-preserving key << 32) | ~index, so that a larger word means a larger
 // value or, for equal values, a lower index.
+// Four CTAs per SM (registers capped at 32), so the 512 CTAs of 64 long rows
+// run as one wave.
 template <int C, int NT, int EPT>
-__global__ void __launch_bounds__(NT) topk_cluster_kernel(TopkArgs a)
+__global__ void __launch_bounds__(NT, 4) topk_cluster_kernel(TopkArgs a)
 {
     constexpr int G = EPT / 4;                  // float4 groups per thread
     constexpr int PER_T = kCBuckets / NT;        // buckets per thread in the scan

@@ -14,7 +14,8 @@ namespace li {
 constexpr int kTileKeys = 128;        // keys per MMA tile (the M axis)
 constexpr int kAccCols = 256;         // TMEM columns per accumulator (the N axis)
 constexpr int kAccStages = 2;         // double-buffered accumulators (512 TMEM columns)
-constexpr int kEpiWarps = 8;          // epilogue warps (2 per TMEM lane quarter)
+constexpr int kGroupWarps = 8;        // warps of one epilogue group (2 per TMEM lane quarter)
+constexpr int kEpiWarps = kAccStages * kGroupWarps;   // one group per accumulator
 constexpr int kQCost = 2;             // scheduler weight of one query-tile load, in key tiles
 constexpr int kScoreThreads = 32 * (2 + kEpiWarps);
 constexpr int kTopkThreads = 512;

@@ -120,21 +120,6 @@ __device__ __forceinline__ void unpack2(uint64_t r, float &lo, float &hi)
     asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
 }
 
-// s32 accumulator bits (as loaded from TMEM) to fp32, in place.  Exact for
-// |x| < 2^22 (an int8 dot product over D = 128 is at most 2^21): the bit
-// pattern of 1.5*2^23 plus x is the float 1.5*2^23 + x, and subtracting
-// 1.5*2^23 leaves x.
-__device__ __forceinline__ void s32_to_f32(float (&v)[32])
-{
-    const uint64_t m2 = pack2(-12582912.f, -12582912.f);
-#pragma unroll
-    for (int i = 0; i < 32; i += 2) {
-        const float a = __int_as_float(__float_as_int(v[i]) + 0x4B400000);
-        const float b = __int_as_float(__float_as_int(v[i + 1]) + 0x4B400000);
-        unpack2(fadd2(pack2(a, b), m2), v[i], v[i + 1]);
-    }
-}
-
 __device__ __forceinline__ float hsum2(uint64_t r)
 {
     float lo, hi;
@@ -158,29 +143,32 @@ __device__ __forceinline__ float relu_c(float x)
     else return fmaxf(x, 0.f);
 }
 
-template <int C, int J, int QPW, int NP2, int N1P>
-__device__ __forceinline__ void epi_group(const float (&v)[32], const uint4 ww, uint64_t (&part)[QPW][NP2])
+// Four columns COL0..COL0+3 of the warp's 128: W * ReLU(logit) accumulated
+// into the packed partial sums of their query.
+template <int COL0, int QPW, int NP2, int N1P>
+__device__ __forceinline__ void epi_quad(const float *v, const uint4 ww, uint64_t (&part)[QPW][NP2])
 {
-    constexpr int q = (C * 32 + J) / N1P;
-    constexpr int p0 = (J / 2) % NP2, p1 = (J / 2 + 1) % NP2;
+    constexpr int q = COL0 / N1P;
+    constexpr int p0 = (COL0 / 2) % NP2, p1 = (COL0 / 2 + 1) % NP2;
     const uint64_t w01 = pack2(__uint_as_float(ww.x), __uint_as_float(ww.y));
     const uint64_t w23 = pack2(__uint_as_float(ww.z), __uint_as_float(ww.w));
-    part[q][p0] = ffma2(w01, pack2(relu_c<C * 32 + J>(v[J]), relu_c<C * 32 + J + 1>(v[J + 1])), part[q][p0]);
-    part[q][p1] = ffma2(w23, pack2(relu_c<C * 32 + J + 2>(v[J + 2]), relu_c<C * 32 + J + 3>(v[J + 3])), part[q][p1]);
+    part[q][p0] = ffma2(w01, pack2(relu_c<COL0>(v[0]), relu_c<COL0 + 1>(v[1])), part[q][p0]);
+    part[q][p1] = ffma2(w23, pack2(relu_c<COL0 + 2>(v[2]), relu_c<COL0 + 3>(v[3])), part[q][p1]);
 }
 
-template <int C, int QPW, int NP2, int N1P>
-__device__ __forceinline__ void epi_chunk(const float (&v)[32], const float *myW, uint64_t (&part)[QPW][NP2])
+// s32 accumulator bits to fp32, in place; exact for |x| < 2^22 (an int8 dot
+// product over D = 128 is at most 2^21): the bit pattern of 1.5*2^23 plus x
+// is the float 1.5*2^23 + x, and subtracting 1.5*2^23 leaves x.
+__device__ __forceinline__ void s32_to_f32_16(uint32_t (&r)[16])
 {
-    const uint4 *w4 = reinterpret_cast<const uint4 *>(myW + C * 32);
-    epi_group<C, 0, QPW, NP2, N1P>(v, w4[0], part);
-    epi_group<C, 4, QPW, NP2, N1P>(v, w4[1], part);
-    epi_group<C, 8, QPW, NP2, N1P>(v, w4[2], part);
-    epi_group<C, 12, QPW, NP2, N1P>(v, w4[3], part);
-    epi_group<C, 16, QPW, NP2, N1P>(v, w4[4], part);
-    epi_group<C, 20, QPW, NP2, N1P>(v, w4[5], part);
-    epi_group<C, 24, QPW, NP2, N1P>(v, w4[6], part);
-    epi_group<C, 28, QPW, NP2, N1P>(v, w4[7], part);
+    const uint64_t m2 = pack2(-12582912.f, -12582912.f);
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+        float lo, hi;
+        unpack2(fadd2(pack2(__uint_as_float(r[i] + 0x4B400000u), __uint_as_float(r[i + 1] + 0x4B400000u)), m2), lo, hi);
+        r[i] = __float_as_uint(lo);
+        r[i + 1] = __float_as_uint(hi);
+    }
 }
 
 __device__ __forceinline__ void release_acc(uint64_t *bar, int lane)
@@ -190,44 +178,42 @@ __device__ __forceinline__ void release_acc(uint64_t *bar, int lane)
     if (lane == 0) mbar_arrive(bar);
 }
 
-// Loads the warp's columns from TMEM two 32-column chunks at a time and
-// reduces them into `part`; hands the accumulator back to the MMA warp once
-// every column is in registers.  NFULL = 4 is the common case of a full query
-// block (no runtime chunk checks); NFULL = 0 takes the chunk count at run time.
-template <int QPW, int NP2, int N1P, int NFULL, int KIND>
-__device__ __forceinline__ void epi_reduce(uint32_t trow, int nchunks, const float *myW,
+// 16-column chunk C of the warp's 128 columns.  The chunk's TMEM load was
+// issued into `cur` by the previous step; this step waits for it, issues the
+// next chunk's load into `nxt` (or, after the last load, hands the
+// accumulator back to the MMA warp), then reduces `cur` while the next load
+// is in flight.
+template <int C, int QPW, int NP2, int N1P, int KIND>
+__device__ __forceinline__ void epi_step(uint32_t trow, int nc, const float *myW,
+                                         uint64_t (&part)[QPW][NP2], uint64_t *bar, int lane,
+                                         uint32_t (&cur)[16], uint32_t (&nxt)[16])
+{
+    if constexpr (C < 8) {
+        if (C >= nc) return;
+        tmem_ld_wait16(cur);
+        if (C + 1 < nc) tmem_ld16(trow + 16 * (C + 1), nxt);
+        else release_acc(bar, lane);
+        if constexpr (KIND == kKindI8) s32_to_f32_16(cur);
+        const float *v = reinterpret_cast<const float *>(cur);
+        const uint4 *w4 = reinterpret_cast<const uint4 *>(myW + C * 16);
+        epi_quad<C * 16 + 0, QPW, NP2, N1P>(v + 0, w4[0], part);
+        epi_quad<C * 16 + 4, QPW, NP2, N1P>(v + 4, w4[1], part);
+        epi_quad<C * 16 + 8, QPW, NP2, N1P>(v + 8, w4[2], part);
+        epi_quad<C * 16 + 12, QPW, NP2, N1P>(v + 12, w4[3], part);
+        epi_step<C + 1, QPW, NP2, N1P, KIND>(trow, nc, myW, part, bar, lane, nxt, cur);
+    }
+}
+
+// Reduces the warp's columns (nc 16-column chunks, nc >= 1) into `part`,
+// double-buffering the TMEM loads; the accumulator is released as soon as
+// the last chunk is in registers.
+template <int QPW, int NP2, int N1P, int KIND>
+__device__ __forceinline__ void epi_reduce(uint32_t trow, int nc, const float *myW,
                                            uint64_t (&part)[QPW][NP2], uint64_t *bar, int lane)
 {
-    constexpr bool S32 = KIND == kKindI8;       // integer accumulator
-    const int nc = NFULL ? NFULL : nchunks;
-    {
-        float v0[32], v1[32];
-        if (nc > 0) tmem_ld32(trow, v0);
-        if (nc > 1) tmem_ld32(trow + 32, v1);
-        if (nc > 0) {
-            tmem_ld_wait();
-            if (nc <= 2) release_acc(bar, lane);
-            if constexpr (S32) {
-                s32_to_f32(v0);
-                if (nc > 1) s32_to_f32(v1);
-            }
-        }
-        if (nc > 0) epi_chunk<0, QPW, NP2, N1P>(v0, myW, part);
-        if (nc > 1) epi_chunk<1, QPW, NP2, N1P>(v1, myW, part);
-    }
-    if (nc > 2) {
-        float v0[32], v1[32];
-        tmem_ld32(trow + 64, v0);
-        if (nc > 3) tmem_ld32(trow + 96, v1);
-        tmem_ld_wait();
-        release_acc(bar, lane);
-        if constexpr (S32) {
-            s32_to_f32(v0);
-            if (nc > 3) s32_to_f32(v1);
-        }
-        epi_chunk<2, QPW, NP2, N1P>(v0, myW, part);
-        if (nc > 3) epi_chunk<3, QPW, NP2, N1P>(v1, myW, part);
-    }
+    uint32_t b0[16], b1[16];
+    tmem_ld16(trow, b0);
+    epi_step<0, QPW, NP2, N1P, KIND>(trow, nc, myW, part, bar, lane, b0, b1);
 }
 
 __device__ __forceinline__ float load_weight(const void *w, int dtype, int64_t i)
@@ -259,7 +245,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     constexpr int STAGES = G::STAGES;
     constexpr int NQ = 256 / N1P;                 // queries per block
     constexpr int QPW = 128 / N1P;                // queries per epilogue warp half
-    constexpr int NP2 = N1P >= 32 ? 4 : (N1P == 16 ? 2 : 1);  // packed partial sums per query
+    constexpr int NP2 = N1P >= 64 ? 4 : (N1P == 32 ? 2 : 1);  // packed partial sums per query
     constexpr int INNER = KIND == kKindF16 ? 64 : 128;   // elements per 128-byte row chunk
 
     extern __shared__ uint8_t smem_raw[];
@@ -291,7 +277,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         mbar_init(q_empty, 1);
         for (int s = 0; s < kAccStages; ++s) {
             mbar_init(&acc_full[s], 1);
-            mbar_init(&acc_empty[s], kEpiWarps);
+            mbar_init(&acc_empty[s], kGroupWarps);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -516,26 +502,33 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        // Each thread owns key row `lrow` of the tile and the 128 columns of
-        // its warp half: QPW queries x N1P heads.  Per tile it loads those
-        // columns from TMEM in one go, hands the accumulator back to the MMA
-        // warp, then reduces sum_h W*ReLU(logit) with packed fp32 FMAs.
-        const int ew = warp - 2;                   // 0..7
-        const int quarter = warp & 3;              // TMEM lanes this warp may access
-        const int half = ew >> 2;                  // which 128 of the 256 columns
+        // Two groups of eight warps, one per accumulator: group g takes the
+        // tiles of accumulator g (every other tile), so one group reduces a
+        // tile while the other loads the next, and each has two MMA times
+        // per tile.  In a group, each thread owns key row `lrow` of the tile
+        // and the 128 columns of its warp half (QPW queries x N1P heads); it
+        // streams them out of TMEM 16 at a time, hands the accumulator back
+        // once the last chunk is in registers, and reduces
+        // sum_h W*ReLU(logit) with packed fp32 FMAs.
+        const int ew = warp - 2;                   // 0..15
+        const int grp = ew / kGroupWarps;          // the accumulator (tile parity) of this group
+        const int quarter = warp & 3;              // TMEM lane quarter this warp may access
+        const int half = (ew % kGroupWarps) >> 2;  // which 128 of the 256 columns
         const int lrow = quarter * 32 + lane;      // key row within the tile
         float *myW = sW + ew * 128;
         if (w_begin < w_end && nblocks > 0) {
             Walker w{a.blocks, nblocks, 0, 0, 0, 0, 0};
             w.init_from(a.cta_start[blockIdx.x], w_end);
-            int acc = 0, prev_qb = -1, nchunks = 0;
+            const int acc = grp;
+            int prev_qb = -1, nchunks = 0, parity = 0;
             uint32_t acc_phase = 0;
             BlockInfo blk{};
             BatchInfo bi{};
             float *row_ptr = nullptr;              // score row of this half's first query
             int64_t lim0 = 0;                      // visible keys of query q: (lim0 + q) >> cmp_shift
             int nq_valid = 0;                      // valid queries of this warp
-            for (; w.valid(); w.next()) {
+            for (; w.valid(); w.next(), parity ^= 1) {
+                if (parity != grp) continue;       // the other group's tile
                 if (w.qb != prev_qb) {
                     blk = a.blocks[w.qb];
                     bi = a.batches[blk.b];
@@ -544,7 +537,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                     int mine = nrows - half * QPW;     // valid queries of this half
                     mine = mine < 0 ? 0 : (mine > QPW ? QPW : mine);
                     nq_valid = mine;
-                    nchunks = (mine * N1P + 31) / 32;
+                    nchunks = (mine * N1P + 15) / 16;   // 16-column chunks
                     const int i_first = blk.i0 + half * QPW;
                     row_ptr = a.scores + (int64_t)(bi.row0 + i_first) * a.ld;
                     // right-down causal over compressed keys (see causal_visible);
@@ -601,19 +594,16 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 for (int q = 0; q < QPW; ++q)
 #pragma unroll
                     for (int p = 0; p < NP2; ++p) part[q][p] = 0ull;
-                if (nchunks == 4 * QPW * N1P / 128)
-                    epi_reduce<QPW, NP2, N1P, 4, KIND>(trow, 4, myW, part, &acc_empty[acc], lane);
-                else
-                    epi_reduce<QPW, NP2, N1P, 0, KIND>(trow, nchunks, myW, part, &acc_empty[acc], lane);
+                if (nchunks == 8)
+                    epi_reduce<QPW, NP2, N1P, KIND>(trow, 8, myW, part, &acc_empty[acc], lane);
+                else if (nchunks > 0)
+                    epi_reduce<QPW, NP2, N1P, KIND>(trow, nchunks, myW, part, &acc_empty[acc], lane);
                 if (nchunks == 0) {                // nothing to read: release at once
                     tc_fence_before_sync();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&acc_empty[acc]);
                 }
-                if (++acc == kAccStages) {
-                    acc = 0;
-                    acc_phase ^= 1u;
-                }
+                acc_phase ^= 1u;
                 // visible keys only: t < nvis(i); the row keeps its visible prefix
 #pragma unroll
                 for (int q = 0; q < QPW; ++q) {

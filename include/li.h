@@ -218,6 +218,63 @@ LI_API li_status li_indexer_noalloc(const li_params *p, const void *query, const
                                     const int32_t *act_seq_k, const int32_t *block_table,
                                     int32_t *sparse_indices, float *sparse_values, void *stream);
 
+/*
+ * Sparse attention over the selected keys: the consumer of the indexer's
+ * output (CANN TileLang LightningIndexer guide, section "LightningIndexer 在
+ * 稀疏注意力中的地位": an explicit index tensor names, for every query token,
+ * the key/value subset it attends to, so attention costs O(N*S) instead of
+ * O(N^2); the open-sourcing issue, section 3: the forward's sparse_indices feed
+ * Sparse FlashAttention).  The pages give no formula of their own for it; this
+ * library computes scaled dot-product attention restricted to each row's
+ * selected keys, with one key/value head shared by all query heads:
+ *
+ *     J      = entries j of the row's index list with 0 <= j < Sk_b
+ *     out_h  = sum_{j in J} softmax_j(scale * q_h . k_j) * v_j
+ *     lse_h  = log sum_{j in J} exp(scale * q_h . k_j)
+ *
+ * and out = 0, lse = -inf for rows with J empty and for BSND padding rows.
+ *
+ *   layout_q       LI_BSND: query/out [B,S1,N1,D]; LI_TND: [T1,N1,D]
+ *   layout_kv      LI_BSND: key [B,S2,1,D], value [B,S2,1,Dv]; LI_TND: [T2,1,D] /
+ *                  [T2,1,Dv]; LI_PA_BSND: [num_blocks,block_size,1,D] / [..,Dv]
+ *                  through block_table (a dense pool)
+ *   dtype          LI_BF16 or LI_FP16 for query, key, value and out
+ *   N1             query heads: 16, 32, 64 or 128
+ *   D, Dv          128 and 128
+ *   sparse_count   K, entries per index row, 1..65536
+ *   softmax_scale  > 0 and finite (1/sqrt(D) is the usual choice)
+ *   B, S1, S2, T1, T2, num_blocks, block_size, max_blocks_per_seq  as in li_params
+ *   reserved       must be 0
+ *
+ *   sparse_indices int32 [rows, K] (the indexer's output layout): batch-local
+ *                  key positions; -1 marks an empty slot.  An entry >= Sk_b or
+ *                  below -1 is skipped and flagged with LI_DEV_BAD_INDEX.
+ *   act_seq_q, act_seq_k, block_table   as for li_indexer
+ *   out            [rows, N1, Dv] in dtype (device)
+ *   lse            fp32 [rows, N1] (device) or NULL
+ *   status         device int32 that receives LI_DEV_* bits by atomic OR, or
+ *                  NULL; the caller clears it
+ * Accumulation is fp32 on the tensor cores; the softmax weights enter the P.V
+ * product rounded to dtype.  Needs no workspace.  One launch.
+ */
+#define LI_DEV_BAD_INDEX     0x20  /* sparse attention: an index outside [-1, Sk) (skipped) */
+typedef struct {
+    int32_t layout_q, layout_kv;
+    int32_t dtype;
+    int32_t B, S1, S2, T1, T2;
+    int32_t N1, D, Dv;
+    int32_t num_blocks, block_size, max_blocks_per_seq;
+    int32_t sparse_count;
+    float softmax_scale;
+    int32_t reserved;
+} li_sfa_params;
+
+LI_API li_status li_sparse_attention(const li_sfa_params *p, const void *query, const void *key,
+                                     const void *value, const int32_t *sparse_indices,
+                                     const int32_t *act_seq_q, const int32_t *act_seq_k,
+                                     const int32_t *block_table, void *out, float *lse,
+                                     int32_t *status, void *stream);
+
 /* Thread-local message describing the last non-OK status. */
 LI_API const char *li_last_error(void);
 

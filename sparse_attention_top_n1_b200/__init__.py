@@ -26,11 +26,13 @@ STATUS_NAMES = {0: "LI_OK", 1: "LI_ERR_NULL", 2: "LI_ERR_SHAPE", 3: "LI_ERR_DTYP
 DTYPE = {"bf16": 0, "fp16": 1, "fp32": 2, "e4m3": 3, "int8": 4}
 LAYOUT = {"BSND": 0, "TND": 1, "PA_BSND": 2}
 DEV_BAD_QLEN, DEV_BAD_KLEN, DEV_BAD_BLOCK, DEV_NEG_SCALE, DEV_TIMEOUT = 1, 2, 4, 8, 16
+DEV_BAD_INDEX = 32
 INT64_MAX = (1 << 63) - 1
 
 EXPORTS = ("li_output_shape", "li_workspace_size", "li_indexer", "li_quant_indexer", "li_topk",
            "li_last_error", "li_read_device_status", "li_selftest_bounded_wait",
-           "li_last_launch_count", "li_set_profile_events", "li_indexer_noalloc")
+           "li_last_launch_count", "li_set_profile_events", "li_indexer_noalloc",
+           "li_sparse_attention")
 
 
 class LiError(RuntimeError):
@@ -60,6 +62,19 @@ class Params(ctypes.Structure):
     ]
 
 
+class SfaParams(ctypes.Structure):
+    """Mirror of li_sfa_params (sparse attention over the selected keys)."""
+    _fields_ = [
+        ("layout_q", ctypes.c_int32), ("layout_kv", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("B", ctypes.c_int32), ("S1", ctypes.c_int32), ("S2", ctypes.c_int32),
+        ("T1", ctypes.c_int32), ("T2", ctypes.c_int32),
+        ("N1", ctypes.c_int32), ("D", ctypes.c_int32), ("Dv", ctypes.c_int32),
+        ("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32),
+        ("max_blocks_per_seq", ctypes.c_int32), ("sparse_count", ctypes.c_int32),
+        ("softmax_scale", ctypes.c_float), ("reserved", ctypes.c_int32),
+    ]
+
+
 _lib = None
 
 
@@ -84,6 +99,8 @@ def lib() -> ctypes.CDLL:
             "li_last_launch_count": (i32, []),
             "li_set_profile_events": (None, [ctypes.POINTER(ctypes.c_void_p), i32]),
             "li_indexer_noalloc": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+            "li_sparse_attention": (ctypes.c_int, [ctypes.POINTER(SfaParams), vp, vp, vp, vp, vp,
+                                                   vp, vp, vp, vp, vp, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -184,6 +201,46 @@ def li_indexer_noalloc(params, query, key, weights, act_seq_q, act_seq_k, block_
     _check(lib().li_indexer_noalloc(ctypes.byref(params), _ptr(query), _ptr(key), _ptr(weights),
                                     _ptr(act_seq_q), _ptr(act_seq_k), _ptr(block_table),
                                     _ptr(sparse_indices), _ptr(sparse_values), _stream(stream)))
+
+
+def make_sfa_params(problem=None, **kw) -> SfaParams:
+    """li_sfa_params from an object with its field names (layouts and dtype as
+    strings; softmax_scale 0 or absent = 1/sqrt(D)) and/or keyword overrides."""
+    f = {}
+    if problem is not None:
+        for name, _ in SfaParams._fields_:
+            if hasattr(problem, name):
+                f[name] = getattr(problem, name)
+    f.update(kw)
+    for name in ("layout_q", "layout_kv"):
+        if isinstance(f.get(name), str):
+            f[name] = LAYOUT[f[name]]
+    if isinstance(f.get("dtype"), str):
+        f["dtype"] = DTYPE[f["dtype"]]
+    if not f.get("softmax_scale"):
+        f["softmax_scale"] = f.get("D", 128) ** -0.5
+    return SfaParams(**{k: v for k, v in f.items() if k in dict(SfaParams._fields_)})
+
+
+def li_sparse_attention(params: SfaParams, query, key, value, sparse_indices, act_seq_q, act_seq_k,
+                        block_table, out, lse=None, status=None, stream=None):
+    _check(lib().li_sparse_attention(ctypes.byref(params), _ptr(query), _ptr(key), _ptr(value),
+                                     _ptr(sparse_indices), _ptr(act_seq_q), _ptr(act_seq_k),
+                                     _ptr(block_table), _ptr(out), _ptr(lse), _ptr(status),
+                                     _stream(stream)))
+
+
+def sparse_attention(params: SfaParams, query, key, value, sparse_indices, *, act_seq_q=None,
+                     act_seq_k=None, block_table=None, want_lse=True, status=None, stream=None):
+    """Run li_sparse_attention, allocating out [rows, N1, Dv] (the query's dtype)
+    and, when asked, lse [rows, N1] fp32.  Returns (out, lse or None)."""
+    import torch
+    rows = params.B * params.S1 if params.layout_q == LAYOUT["BSND"] else params.T1
+    out = torch.empty((rows, params.N1, params.Dv), dtype=query.dtype, device=query.device)
+    lse = torch.empty((rows, params.N1), dtype=torch.float32, device=query.device) if want_lse else None
+    li_sparse_attention(params, query, key, value, sparse_indices, act_seq_q, act_seq_k, block_table,
+                        out, lse, status, stream)
+    return out, lse
 
 
 def li_read_device_status(workspace, stream=None) -> int:

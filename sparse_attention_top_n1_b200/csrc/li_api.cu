@@ -426,6 +426,7 @@ namespace li {
 // Record `msg` as the thread's last error and return `s` (for the other
 // translation units of the library).
 li_status report_error(li_status s, const char *msg) { return fail(s, "%s", msg); }
+void set_launch_count(int32_t n) { g_launches = n; }
 }  // namespace li
 
 extern "C" {

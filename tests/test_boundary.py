@@ -206,3 +206,71 @@ def test_oracle_and_cuda_path_share_no_source():
         assert "oracle" not in txt.lower(), f
     pkg = open(os.path.join(ROOT, "sparse_attention_top_n1_b200", "__init__.py")).read()
     assert "import oracle" not in pkg and "from oracle" not in pkg
+
+
+# ---------------------------------------------------------------- sparse attention
+
+def test_sfa_params_struct_matches_header_layout(tmp_path):
+    fields = [name for name, _ in li.SfaParams._fields_]
+    src = tmp_path / "probe_sfa.c"
+    src.write_text("#include <stdio.h>\n#include <stddef.h>\n#include \"li.h\"\n"
+                   "int main(void) {\n  printf(\"%zu\\n\", sizeof(li_sfa_params));\n" +
+                   "".join('  printf("%%zu\\n", offsetof(li_sfa_params, %s));\n' % f for f in fields) +
+                   "  return 0;\n}\n")
+    exe = tmp_path / "probe_sfa"
+    subprocess.check_call(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)])
+    out = [int(x) for x in subprocess.check_output([str(exe)]).split()]
+    assert out[0] == ctypes.sizeof(li.SfaParams)
+    for f, off in zip(fields, out[1:]):
+        assert getattr(li.SfaParams, f).offset == off, f
+
+
+def _sfa_base(**kw):
+    f = dict(layout_q="BSND", layout_kv="BSND", dtype="bf16", B=2, S1=16, S2=64, N1=64, D=128,
+             Dv=128, sparse_count=32)
+    f.update(kw)
+    return li.make_sfa_params(**f)
+
+
+@pytest.mark.parametrize("kw,err", [
+    (dict(N1=48), "LI_ERR_SHAPE"), (dict(N1=256), "LI_ERR_SHAPE"),
+    (dict(D=64), "LI_ERR_UNSUPPORTED"), (dict(Dv=256), "LI_ERR_UNSUPPORTED"),
+    (dict(dtype="fp32"), "LI_ERR_DTYPE"), (dict(dtype="e4m3"), "LI_ERR_DTYPE"),
+    (dict(sparse_count=0), "LI_ERR_SHAPE"), (dict(sparse_count=65537), "LI_ERR_SHAPE"),
+    (dict(softmax_scale=-1.0), "LI_ERR_SHAPE"), (dict(softmax_scale=float("inf")), "LI_ERR_SHAPE"),
+    (dict(reserved=1), "LI_ERR_SHAPE"), (dict(layout_kv="TND"), "LI_ERR_LAYOUT"),
+    (dict(layout_q="PA_BSND"), "LI_ERR_LAYOUT"), (dict(B=0), "LI_ERR_SHAPE"),
+    (dict(S1=-1), "LI_ERR_SHAPE"), (dict(B=70000, S2=70000), "LI_ERR_SHAPE"),
+])
+def test_sfa_rejects_before_launch(kw, err):
+    pr = _sfa_base(**kw)
+    st = li.lib().li_sparse_attention(ctypes.byref(pr), FAKE, FAKE, FAKE, FAKE, None, None, None,
+                                      FAKE, None, None, None)
+    assert li.STATUS_NAMES[st] == err, li.li_last_error()
+
+
+def test_sfa_pointer_checks():
+    L = li.lib()
+    pr = _sfa_base()
+    call = lambda q=FAKE, k=FAKE, v=FAKE, i=FAKE, aq=None, ak=None, bt=None, o=FAKE, lse=None, p=pr: \
+        li.STATUS_NAMES[L.li_sparse_attention(ctypes.byref(p), q, k, v, i, aq, ak, bt, o, lse, None, None)]
+    assert call(q=None) == "LI_ERR_NULL"
+    assert call(v=None) == "LI_ERR_NULL"
+    assert call(i=None) == "LI_ERR_NULL"
+    assert call(o=None) == "LI_ERR_NULL"
+    assert call(k=FAKE + 8) == "LI_ERR_SHAPE"           # 16-byte alignment
+    assert call(o=FAKE + 4) == "LI_ERR_SHAPE"
+    tnd = _sfa_base(layout_q="TND", layout_kv="TND", T1=8, T2=8)
+    assert call(p=tnd) == "LI_ERR_NULL"                  # TND needs the prefix sums
+    pa = _sfa_base(layout_kv="PA_BSND", num_blocks=4, block_size=16, max_blocks_per_seq=2)
+    assert call(p=pa, ak=FAKE) == "LI_ERR_NULL"          # PA needs the block table
+    assert call(p=_sfa_base(S1=0)) == "LI_OK"            # nothing to do, nothing launched
+    assert li.li_last_launch_count() == 0
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_sfa_valid_call_without_device_reports_cuda_error():
+    pr = _sfa_base()
+    st = li.lib().li_sparse_attention(ctypes.byref(pr), FAKE, FAKE, FAKE, FAKE, None, None, None,
+                                      FAKE, None, None, None)
+    assert li.STATUS_NAMES[st] == "LI_ERR_CUDA"

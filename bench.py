@@ -4,7 +4,9 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 One step is one full indexer call (all three kernels) over one batch of the
-named synthetic workload, with inputs resident in HBM.  The default workload
+named synthetic workload, with inputs resident in HBM.  The ``sfa_*``
+workloads instead time one call of the sparse attention consumer
+(li_sparse_attention) over its own synthetic inputs.  The default workload
 is the TileLang test shape (B=2, S1=512, S2=4096, G=32, D=64, k=1024, fp16,
 no mask).  L2 is flushed before every timed step (a 256 MiB device write,
 then a 256 MiB read of a second buffer so no dirty lines are left behind),
@@ -51,7 +53,11 @@ WORKLOAD_DESC = {
     "quant_varlen_int8": "quant varlen TND {2k,4k,8k,16k} N1=64 D=128 int8 + fp16 scales/weights, k=2048 mode3",
     "quant_int8_pa": "quant int8 PA (VllmQuant README A3 example): B=24 S1=4 S2=512 N1=64 D=128 block 128, fp16 scales/weights, k=512 mode0",
     "dsa_prefill_window": "DSA prefill with sink/local window: B=1 S1=S2=8192 N1=64 D=128 k=2048 mode3 bf16, init_num=16 local_num=512, values on",
+    "sfa_prefill": "sparse attention consumer of DSA prefill: 8192 rows x 64 heads, K=2048 selected keys (causal), D=Dv=128 bf16",
+    "sfa_decode": "sparse attention consumer of paged decode: 64 rows x 64 heads over a PA pool (block 128, lengths U[4096,65536]), K=2048, D=Dv=128 bf16",
 }
+SFA_METRIC = "sparse attention query rows/s at 1 B200 (the indexer's consumer); % of tensor roofline"
+SFA_UNIT = "rows/s"
 RETURN_VALUE = {"tiny": 1, "cfg2": 1, "dsa_prefill": 1, "paged_decode": 0, "quant_varlen": 0,
                 "quant_varlen_int8": 0, "quant_int8_pa": 0, "dsa_prefill_window": 1}
 
@@ -290,6 +296,185 @@ def run_reference(args, ws, rank):
     return 0
 
 
+def blas_threads():
+    """Threads the numpy oracle's matrix products may use (its BLAS pool)."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def sfa_workload(name):
+    from synth import sfa as ssfa
+    return ssfa.make_sfa_prefill() if name == "sfa_prefill" else ssfa.make_sfa_decode()
+
+
+def sfa_counts(p, inp):
+    """Valid (row, selected key) pairs, FLOPs and gathered bytes of one call."""
+    idx = inp["sparse_indices"].reshape(p.rows, p.sparse_count)
+    pairs = int((idx >= 0).sum())
+    flops = 2.0 * p.N1 * (p.D + p.Dv) * pairs
+    gathered = pairs * (p.D + p.Dv) * 2
+    io = p.rows * p.N1 * (p.D + p.Dv) * 2 + idx.numel() * 4 + p.rows * p.N1 * 4
+    return pairs, flops, gathered, io
+
+
+def sfa_reference(args, rank):
+    """Reference arm for the sparse attention workloads: the fp64 oracle on
+    bounded row samples on the host cores."""
+    if rank != 0:
+        return 0
+    import numpy as np
+
+    import oracle.sfa as osfa
+    p, inp = sfa_workload(args.workload)
+    rng = np.random.default_rng(1)
+    probe = sorted(rng.choice(p.rows, size=min(p.rows, 8), replace=False).tolist())
+    t0 = time.perf_counter()
+    osfa.run(p, inp, rows=probe)
+    per_row = (time.perf_counter() - t0) / len(probe)
+    total_steps = args.steps + args.warmup
+    step_budget = max(0.5, min(6.0, 150.0 / max(total_steps, 1)))
+    n = int(min(p.rows, max(2, step_budget / max(per_row, 1e-9))))
+    times = []
+    for st in range(total_steps):
+        rows = sorted(rng.choice(p.rows, size=n, replace=False).tolist())
+        t0 = time.perf_counter()
+        osfa.run(p, inp, rows=rows)
+        if st >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    tot = sum(times)
+    value = n * len(times) / tot
+    line = {"metric": SFA_METRIC, "value": value, "unit": SFA_UNIT, "impl": "reference", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD_DESC[args.workload], "rows_per_step": n},
+            "cpu_baseline": {"value": value, "unit": SFA_UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": "%d of %d rows per step, fp64 numpy oracle" % (n, p.rows)},
+            "e2e": {"value": value, "unit": SFA_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def sfa_main(args, ws, rank, local):
+    """One step = one li_sparse_attention call over the whole workload."""
+    import torch
+
+    import sparse_attention_top_n1_b200 as li
+    from sparse_attention_top_n1_b200 import build as libbuild
+    if not os.path.exists(li.LIB_PATH):
+        libbuild.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    p, inp = sfa_workload(args.workload)
+    pairs, flops, gathered, io = sfa_counts(p, inp)
+    d = {k: v.to(dev) for k, v in inp.items()}
+    pr = li.make_sfa_params(p)
+    out = torch.empty((p.rows, p.N1, p.Dv), dtype=d["query"].dtype, device=dev)
+    lse = torch.empty((p.rows, p.N1), dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    clean = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        flush.zero_()
+        clean.sum()
+
+    def call():
+        li.li_sparse_attention(pr, d["query"], d["key"], d["value"], d["sparse_indices"], d.get("act_q"),
+                               d.get("act_k"), d.get("block_table"), out, lse, status)
+
+    clocks = ClockSampler(local)
+    if not args.plain:
+        clocks.start()
+    t_warm = time.perf_counter()
+    nw = 0
+    while nw < args.warmup or (not args.plain and time.perf_counter() - t_warm < 0.8):
+        flush_l2()
+        call()
+        nw += 1
+    torch.cuda.synchronize()
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    K = args.steps
+    st_ev = [mk() for _ in range(K)]
+    en_ev = [mk() for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize()
+    launches = 0
+    for s_ in range(K):
+        flush_l2()
+        st_ev[s_].record()
+        call()
+        en_ev[s_].record()
+        launches += li.li_last_launch_count()
+    torch.cuda.synchronize()
+    barrier()
+    own = sum(st_ev[s_].elapsed_time(en_ev[s_]) for s_ in range(K))
+    total_ms = allreduce_max(own)
+    clk = clocks.stop()
+    if int(status.item()):
+        raise SystemExit("device status 0x%x" % int(status.item()))
+    peaks, peak_src = load_peaks()
+    ms = total_ms / K
+    tflops = flops / (ms * 1e-3) / 1e12
+    roof = {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": tflops / peaks["bf16_tflops"], "traffic": None, "kernel": "sfa",
+            "peak_source": "bf16 burst peak (tcgen05 cuBLAS), %s; this kernel issues m16n8k16 mma.sync" % peak_src}
+    e2e = None
+    if not (args.no_e2e or args.plain):
+        host = {k: v.pin_memory() for k, v in inp.items()}
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = hout.numel() * hout.element_size()
+        e_st = [mk() for _ in range(K + args.warmup)]
+        e_en = [mk() for _ in range(K + args.warmup)]
+        for s_ in range(K + args.warmup):
+            flush_l2()
+            e_st[s_].record()
+            for k2, v in host.items():
+                d[k2].copy_(v, non_blocking=True)
+            call()
+            hout.copy_(out, non_blocking=True)
+            e_en[s_].record()
+        torch.cuda.synchronize()
+        e_ms = allreduce_max(sum(e_st[s_].elapsed_time(e_en[s_]) for s_ in range(args.warmup, K + args.warmup)))
+        e2e = {"value": ws * p.rows * K / (e_ms * 1e-3), "unit": SFA_UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h}
+    cpu = None
+    if rank == 0 and ws == 1 and not (args.no_cpu_baseline or args.plain):
+        import numpy as np
+
+        import oracle.sfa as osfa
+        rng = np.random.default_rng(0)
+        probe = sorted(rng.choice(p.rows, size=min(p.rows, 8), replace=False).tolist())
+        t0 = time.perf_counter()
+        osfa.run(p, inp, rows=probe)
+        per = (time.perf_counter() - t0) / len(probe)
+        n = int(min(p.rows, max(1, 12.0 / max(per, 1e-9))))
+        rows = sorted(rng.choice(p.rows, size=n, replace=False).tolist())
+        t0 = time.perf_counter()
+        osfa.run(p, inp, rows=rows)
+        dt = time.perf_counter() - t0
+        cpu = {"value": n / dt, "unit": SFA_UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": "%d of %d rows (seeded uniform sample), fp64 numpy oracle, %.2f s" % (n, p.rows, dt)}
+    line = {
+        "metric": SFA_METRIC, "value": ws * p.rows * K / (total_ms * 1e-3), "unit": SFA_UNIT, "n_gpus": ws,
+        "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD_DESC[args.workload], "rows": p.rows, "selected_pairs": pairs,
+                   "l2": "flushed before every timed step (256 MiB write, then a 256 MiB read of a second buffer)",
+                   "parallelism": "independent replica per GPU" if ws > 1 else "1 GPU"},
+        "effective_tflops": tflops,
+        "gathered_gbs": gathered / (ms * 1e-3) / 1e9,
+        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -308,6 +493,12 @@ def main():
     args.warmup = max(args.warmup, 3)
 
     ws, rank, local = dist_setup()
+    if args.workload.startswith("sfa_"):
+        rc = sfa_reference(args, rank) if args.impl == "reference" else sfa_main(args, ws, rank, local)
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return rc
     if args.impl == "reference":
         rc = run_reference(args, ws, rank)
         if ws > 1:

@@ -19,6 +19,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+#include <cooperative_groups.h>
 
 #include <cmath>
 #include <cstdio>
@@ -38,7 +39,8 @@ constexpr int kHd = 128;                  // D = Dv
 constexpr int kRowBytes = kHd * 2;        // one key or value row
 constexpr int kChunks = kRowBytes / 16;   // 16-byte chunks per row
 constexpr int kTileBytes = kTile * kRowBytes;
-constexpr int kSmem = 4 * kTileBytes + 2 * kTile * 4 + 128;
+constexpr int kSmem = 4 * kTileBytes + 2 * kTile * 4 + 2 * 128 * 4 + 128;
+constexpr int kMaxSplit = 8;             // CTAs (one cluster) sharing a row's keys
 
 struct SfaArgs {
     const uint16_t *q, *k, *v;
@@ -123,7 +125,10 @@ __device__ __forceinline__ int32_t clampi(int64_t v, int64_t lo, int64_t hi)
     return (int32_t)(v < lo ? lo : (v > hi ? hi : v));
 }
 
-template <int NW, bool F16>
+// C > 1: a cluster of C CTAs shares one row; CTA `part` takes its share of the
+// row's key tiles, and the C partial (max, sum, O) triples are merged through
+// distributed shared memory, so no global scratch is needed.
+template <int NW, bool F16, int C>
 __global__ void __launch_bounds__(32 * NW) sfa_kernel(const SfaArgs a)
 {
     static_assert(kChunks == 16, "row chunk arithmetic assumes 256-byte rows");
@@ -136,7 +141,8 @@ __global__ void __launch_bounds__(32 * NW) sfa_kernel(const SfaArgs a)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, c = lane & 3;
-    const int row = blockIdx.x;
+    const int row = blockIdx.x / C;
+    const int part = C > 1 ? (int)(blockIdx.x % C) : 0;   // rank in the cluster
 
     // ---- the row's batch, its position and the batch's keys
     int b = 0, i = 0, Sq = 0;
@@ -230,17 +236,18 @@ __global__ void __launch_bounds__(32 * NW) sfa_kernel(const SfaArgs a)
     for (int dn = 0; dn < 16; ++dn) o[dn][0] = o[dn][1] = o[dn][2] = o[dn][3] = 0.f;
     float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
 
-    const int ntiles = valid_row ? (a.K + kTile - 1) / kTile : 0;
+    const int nt_all = valid_row ? (a.K + kTile - 1) / kTile : 0;
+    const int t_begin = nt_all * part / C, t_end = nt_all * (part + 1) / C;
     int any_cur = 0;
-    if (ntiles > 0) {
-        any_cur = __syncthreads_or(resolve(0, 0));
+    if (t_begin < t_end) {
+        any_cur = __syncthreads_or(resolve(t_begin, 0));
         if (any_cur) issue(0);
         else cp_async_commit();
     }
-    for (int t = 0; t < ntiles; ++t) {
-        const int buf = t & 1;
+    for (int t = t_begin; t < t_end; ++t) {
+        const int buf = (t - t_begin) & 1;
         int any_next = 0;
-        if (t + 1 < ntiles) {
+        if (t + 1 < t_end) {
             any_next = __syncthreads_or(resolve(t + 1, buf ^ 1));
             if (any_next) issue(buf ^ 1);
             else cp_async_commit();
@@ -336,6 +343,55 @@ __global__ void __launch_bounds__(32 * NW) sfa_kernel(const SfaArgs a)
         l[h] += __shfl_xor_sync(0xffffffffu, l[h], 1);
         l[h] += __shfl_xor_sync(0xffffffffu, l[h], 2);
     }
+    if constexpr (C > 1) {
+        // partials into this CTA's shared memory (the tile buffers are free)
+        float *sO = reinterpret_cast<float *>(base);                 // [N1][128], unnormalised
+        float *sM = reinterpret_cast<float *>(base + 4 * kTileBytes + 2 * kTile * 4);   // [N1]
+        float *sL = sM + 128;                                        // [N1]
+        const int h0 = warp * 16 + g, h1 = h0 + 8;
+#pragma unroll
+        for (int dn = 0; dn < 16; ++dn) {
+            const int d = dn * 8 + 2 * c;
+            sO[h0 * kHd + d] = o[dn][0];
+            sO[h0 * kHd + d + 1] = o[dn][1];
+            sO[h1 * kHd + d] = o[dn][2];
+            sO[h1 * kHd + d + 1] = o[dn][3];
+        }
+        if (c == 0) {
+            sM[h0] = m[0];
+            sL[h0] = l[0];
+            sM[h1] = m[1];
+            sL[h1] = l[1];
+        }
+        cooperative_groups::cluster_group cl = cooperative_groups::this_cluster();
+        cl.sync();
+        // CTA `part` merges heads [part*N1/C, (part+1)*N1/C) over the C partials
+        const int hpc = a.N1 / C;
+        const float ln2 = 0.69314718055994531f;
+        for (int e = tid; e < hpc * kHd; e += NT) {
+            const int h = part * hpc + e / kHd, d = e % kHd;
+            float M = -INFINITY;
+#pragma unroll
+            for (int r = 0; r < C; ++r) M = fmaxf(M, cl.map_shared_rank(sM, r)[h]);
+            float L = 0.f, O = 0.f;
+            if (M != -INFINITY) {
+#pragma unroll
+                for (int r = 0; r < C; ++r) {
+                    const float mr = cl.map_shared_rank(sM, r)[h];
+                    if (mr == -INFINITY) continue;
+                    const float w = exp2f(mr - M);
+                    L += cl.map_shared_rank(sL, r)[h] * w;
+                    O += cl.map_shared_rank(sO, r)[h * kHd + d] * w;
+                }
+            }
+            const float v = L > 0.f ? O / L : 0.f;
+            a.out[((int64_t)row * a.N1 + h) * kHd + d] =
+                F16 ? __half_as_ushort(__float2half_rn(v)) : __bfloat16_as_ushort(__float2bfloat16_rn(v));
+            if (d == 0 && a.lse) a.lse[(int64_t)row * a.N1 + h] = L > 0.f ? (M + log2f(L)) * ln2 : -INFINITY;
+        }
+        cl.sync();                             // every peer has read this CTA's partials
+        return;
+    }
     const float inv0 = l[0] > 0.f ? 1.f / l[0] : 0.f, inv1 = l[1] > 0.f ? 1.f / l[1] : 0.f;
     uint16_t *orow = a.out + ((int64_t)row * a.N1 + warp * 16) * kHd;
 #pragma unroll
@@ -352,26 +408,59 @@ __global__ void __launch_bounds__(32 * NW) sfa_kernel(const SfaArgs a)
     }
 }
 
-template <int NW, bool F16>
+template <int NW, bool F16, int C>
 cudaError_t launch(const SfaArgs &a, int rows, cudaStream_t s)
 {
-    auto kern = sfa_kernel<NW, F16>;
+    auto kern = sfa_kernel<NW, F16, C>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
-    kern<<<rows, 32 * NW, kSmem, s>>>(a);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)rows * C);
+    cfg.blockDim = dim3(32 * NW);
+    cfg.dynamicSmemBytes = kSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+template <int NW, bool F16>
+cudaError_t launch_split(const SfaArgs &a, int rows, int split, cudaStream_t s)
+{
+    switch (split) {
+    case 1: return launch<NW, F16, 1>(a, rows, s);
+    case 2: return launch<NW, F16, 2>(a, rows, s);
+    case 4: return launch<NW, F16, 4>(a, rows, s);
+    case 8: return launch<NW, F16, 8>(a, rows, s);
+    }
+    return cudaErrorInvalidValue;
 }
 
 template <bool F16>
-cudaError_t launch_nw(const SfaArgs &a, int rows, cudaStream_t s)
+cudaError_t launch_nw(const SfaArgs &a, int rows, int split, cudaStream_t s)
 {
     switch (a.N1) {
-    case 16: return launch<1, F16>(a, rows, s);
-    case 32: return launch<2, F16>(a, rows, s);
-    case 64: return launch<4, F16>(a, rows, s);
-    case 128: return launch<8, F16>(a, rows, s);
+    case 16: return launch_split<1, F16>(a, rows, split, s);
+    case 32: return launch_split<2, F16>(a, rows, split, s);
+    case 64: return launch_split<4, F16>(a, rows, split, s);
+    case 128: return launch_split<8, F16>(a, rows, split, s);
     }
     return cudaErrorInvalidValue;
+}
+
+// CTAs per row: enough to give every SM two rows' worth of work when rows are
+// few (decode), at least one 64-key tile per CTA, a power of two up to 8.
+int choose_split(int64_t rows, int K, int sms)
+{
+    const int ntiles = (K + kTile - 1) / kTile;
+    int c = 1;
+    while (c < kMaxSplit && rows * c < 2LL * sms && 2 * c <= ntiles) c *= 2;
+    return c;
 }
 
 bool aligned(const void *p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) & (n - 1)) == 0; }
@@ -458,7 +547,11 @@ extern "C" LI_API li_status li_sparse_attention(const li_sfa_params *p, const vo
     a.max_blocks_per_seq = p->max_blocks_per_seq;
     a.scale_log2 = p->softmax_scale * 1.4426950408889634f;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const cudaError_t e = p->dtype == LI_FP16 ? launch_nw<true>(a, (int)rows, s) : launch_nw<false>(a, (int)rows, s);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int split = choose_split(rows, a.K, sms);
+    const cudaError_t e = p->dtype == LI_FP16 ? launch_nw<true>(a, (int)rows, split, s)
+                                              : launch_nw<false>(a, (int)rows, split, s);
     if (e != cudaSuccess) {
         char msg[200];
         snprintf(msg, sizeof msg, "li_sparse_attention: launch failed (%s)", cudaGetErrorString(e));

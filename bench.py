@@ -420,7 +420,7 @@ def sfa_main(args, ws, rank, local):
     ms = total_ms / K
     tflops = flops / (ms * 1e-3) / 1e12
     roof = {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-            "frac": tflops / peaks["bf16_tflops"], "traffic": None, "kernel": "sfa",
+            "frac": tflops / peaks["bf16_tflops"], "traffic": traffic_record(args.workload, "sfa"), "kernel": "sfa",
             "peak_source": "bf16 burst peak (tcgen05 cuBLAS), %s; this kernel issues m16n8k16 mma.sync" % peak_src}
     e2e = None
     if not (args.no_e2e or args.plain):

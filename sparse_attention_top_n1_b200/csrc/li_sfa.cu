@@ -39,7 +39,7 @@ constexpr int kHd = 128;                  // D = Dv
 constexpr int kRowBytes = kHd * 2;        // one key or value row
 constexpr int kChunks = kRowBytes / 16;   // 16-byte chunks per row
 constexpr int kTileBytes = kTile * kRowBytes;
-constexpr int kSmem = 4 * kTileBytes + 2 * kTile * 4 + 2 * 128 * 4 + 128;
+constexpr int kSmem = 4 * kTileBytes + 2 * kTile * 4 + 2 * 128 * 4 + 16 + 128;
 constexpr int kMaxSplit = 8;             // CTAs (one cluster) sharing a row's keys
 
 struct SfaArgs {
@@ -112,6 +112,20 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi)
     }
 }
 
+template <bool F16>
+__device__ __forceinline__ float unpack_lo(uint32_t v)
+{
+    if constexpr (F16) return __half2float(__ushort_as_half((unsigned short)(v & 0xFFFFu)));
+    else return __uint_as_float(v << 16);
+}
+
+template <bool F16>
+__device__ __forceinline__ float unpack_hi(uint32_t v)
+{
+    if constexpr (F16) return __half2float(__ushort_as_half((unsigned short)(v >> 16)));
+    else return __uint_as_float(v & 0xFFFF0000u);
+}
+
 // Byte offset of 16-byte chunk `ch` of row `r` in a tile: rows of 256 B, the
 // low three bits of the chunk index XOR-ed with the row so that the eight
 // rows an ldmatrix phase reads sit in eight different bank groups.
@@ -138,6 +152,7 @@ __global__ void __launch_bounds__(32 * NW) sfa_kernel(const SfaArgs a)
     uint8_t *sK = base;                                      // [2] key tiles
     uint8_t *sV = base + 2 * kTileBytes;                     // [2] value tiles
     int32_t *sRow = reinterpret_cast<int32_t *>(base + 4 * kTileBytes);   // [2][kTile] key row, -1 = none
+    uint32_t *sMask = reinterpret_cast<uint32_t *>(base + 4 * kTileBytes + 2 * kTile * 4 + 2 * 128 * 4);   // [2][2]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, c = lane & 3;
@@ -214,6 +229,9 @@ __global__ void __launch_bounds__(32 * NW) sfa_kernel(const SfaArgs a)
             }
             sRow[buf * kTile + r] = kr;
             ok |= kr >= 0;
+            // whole warps run this loop (kTile is a multiple of 32)
+            const unsigned bal = __ballot_sync(0xffffffffu, kr >= 0);
+            if ((r & 31) == 0) sMask[buf * 2 + (r >> 5)] = bal;
         }
         return ok;
     };
@@ -258,7 +276,7 @@ __global__ void __launch_bounds__(32 * NW) sfa_kernel(const SfaArgs a)
         __syncthreads();
         if (any_cur) {
             const uint32_t kb = smem_addr(sK + buf * kTileBytes), vb = smem_addr(sV + buf * kTileBytes);
-            const int32_t *rmap = sRow + buf * kTile;
+            const uint64_t valid = (uint64_t)sMask[buf * 2] | ((uint64_t)sMask[buf * 2 + 1] << 32);
             // S = Q K^T for 16 heads x 64 keys
             float s[8][4];
 #pragma unroll
@@ -281,7 +299,7 @@ __global__ void __launch_bounds__(32 * NW) sfa_kernel(const SfaArgs a)
             for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const bool ok = rmap[nt * 8 + 2 * c + (e & 1)] >= 0;
+                    const bool ok = (valid >> (nt * 8 + 2 * c + (e & 1))) & 1u;
                     s[nt][e] = ok ? s[nt][e] * a.scale_log2 : -INFINITY;
                     mx[e >> 1] = fmaxf(mx[e >> 1], s[nt][e]);
                 }
@@ -295,33 +313,33 @@ __global__ void __launch_bounds__(32 * NW) sfa_kernel(const SfaArgs a)
                 alpha[h] = exp2f(m[h] - base_[h]);
                 m[h] = mn;
             }
+            // the weights, rounded to dtype as the P.V product sees them, packed
+            // straight into A fragments; the normaliser sums the same values
             float rs[2] = {0.f, 0.f};
+            uint32_t pk[8][2];
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    // the weight as the P.V product will see it (rounded to dtype)
-                    const float p = exp2f(s[nt][e] - base_[e >> 1]);
-                    const float pr = F16 ? __half2float(__float2half_rn(p))
-                                         : __bfloat162float(__float2bfloat16_rn(p));
-                    s[nt][e] = pr;
-                    rs[e >> 1] += pr;
+                for (int h = 0; h < 2; ++h) {
+                    pk[nt][h] = pack2<F16>(exp2f(s[nt][2 * h] - base_[h]), exp2f(s[nt][2 * h + 1] - base_[h]));
+                    rs[h] += unpack_lo<F16>(pk[nt][h]) + unpack_hi<F16>(pk[nt][h]);
                 }
 #pragma unroll
             for (int h = 0; h < 2; ++h) l[h] = l[h] * alpha[h] + rs[h];
+            // the running max moved for some head of this warp: rescale O
+            if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
 #pragma unroll
-            for (int dn = 0; dn < 16; ++dn) {
-                o[dn][0] *= alpha[0];
-                o[dn][1] *= alpha[0];
-                o[dn][2] *= alpha[1];
-                o[dn][3] *= alpha[1];
+                for (int dn = 0; dn < 16; ++dn) {
+                    o[dn][0] *= alpha[0];
+                    o[dn][1] *= alpha[0];
+                    o[dn][2] *= alpha[1];
+                    o[dn][3] *= alpha[1];
+                }
             }
             // O += P V
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const uint32_t pa[4] = {pack2<F16>(s[2 * j][0], s[2 * j][1]), pack2<F16>(s[2 * j][2], s[2 * j][3]),
-                                        pack2<F16>(s[2 * j + 1][0], s[2 * j + 1][1]),
-                                        pack2<F16>(s[2 * j + 1][2], s[2 * j + 1][3])};
+                const uint32_t pa[4] = {pk[2 * j][0], pk[2 * j][1], pk[2 * j + 1][0], pk[2 * j + 1][1]};
 #pragma unroll
                 for (int dp = 0; dp < 8; ++dp) {
                     const int key = j * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);

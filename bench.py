@@ -230,6 +230,19 @@ def barrier():
         dist.barrier()
 
 
+def cpu_model():
+    """The host CPU's model name (for the CPU baseline record)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def cpu_oracle_sample(p, inp, budget_s=12.0, max_rows=None, seed=0):
     """Time the fp64 oracle on a bounded sample of query rows (host cores)."""
     import numpy as np
@@ -250,6 +263,7 @@ def cpu_oracle_sample(p, inp, budget_s=12.0, max_rows=None, seed=0):
     oracle.run(p, inp, rows=rows, nthreads=nthreads)
     dt = time.perf_counter() - t0
     return {"value": len(rows) / dt, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+            "cpu_model": cpu_model(), "nproc": os.cpu_count(),
             "sample": "%d of %d query rows (seeded uniform sample), fp64 C oracle, %.2f s"
                       % (len(rows), R, dt)}, rows, dt
 
@@ -289,6 +303,7 @@ def run_reference(args, ws, rank):
             "data": "synthetic",
             "config": {"workload": WORKLOAD_DESC[args.workload], "rows_per_step": n},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+                             "cpu_model": cpu_model(), "nproc": os.cpu_count(),
                              "sample": "%d of %d query rows per step, fp64 C oracle" % (n, R)},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -352,6 +367,7 @@ def sfa_reference(args, rank):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": WORKLOAD_DESC[args.workload], "rows_per_step": n},
             "cpu_baseline": {"value": value, "unit": SFA_UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "cpu_model": cpu_model(), "nproc": os.cpu_count(),
                              "sample": "%d of %d rows per step, fp64 numpy oracle" % (n, p.rows)},
             "e2e": {"value": value, "unit": SFA_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -458,6 +474,7 @@ def sfa_main(args, ws, rank, local):
         osfa.run(p, inp, rows=rows)
         dt = time.perf_counter() - t0
         cpu = {"value": n / dt, "unit": SFA_UNIT, "cores": blas_threads(), "kind": "oracle",
+               "cpu_model": cpu_model(), "nproc": os.cpu_count(),
                "sample": "%d of %d rows (seeded uniform sample), fp64 numpy oracle, %.2f s" % (n, p.rows, dt)}
     line = {
         "metric": SFA_METRIC, "value": ws * p.rows * K / (total_ms * 1e-3), "unit": SFA_UNIT, "n_gpus": ws,

@@ -8,13 +8,16 @@
 //     out_h = sum_{j in J} softmax_j(scale * q_h . k_j) * v_j,   J = valid entries
 //     lse_h = log sum_{j in J} exp(scale * q_h . k_j)
 //
-// One CTA per query row, one warp per 16 heads.  The row's selected keys are
-// taken 64 at a time: their K and V rows are gathered from wherever the index
-// points (BSND, TND or a paged pool) into shared memory with 16-byte cp.async
-// copies, double-buffered against the math; S = Q K^T and O += P V run on the
-// tensor cores (m16n8k16, fp32 accumulation) with the softmax kept online in
-// registers (running max and sum per head, the FlashAttention recurrence), so
-// the selected keys are read once and nothing but the output is written.
+// One CTA per query row (or, when rows are few, a cluster of up to 8 CTAs per
+// row, each taking a share of its keys), one warp per 16 heads.  The row's
+// selected keys are taken 64 at a time: their K and V rows are gathered from
+// wherever the index points (BSND, TND or a paged pool) into shared memory
+// with 16-byte cp.async copies, double-buffered against the math; S = Q K^T
+// and O += P V run on the tensor cores (m16n8k16, fp32 accumulation) with the
+// softmax kept online in registers (running max and sum per head, the
+// FlashAttention recurrence), so the selected keys are read once and nothing
+// but the output is written.  The weights enter P V rounded to the input
+// type and the normaliser sums the same rounded values.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -39,7 +42,10 @@ constexpr int kHd = 128;                  // D = Dv
 constexpr int kRowBytes = kHd * 2;        // one key or value row
 constexpr int kChunks = kRowBytes / 16;   // 16-byte chunks per row
 constexpr int kTileBytes = kTile * kRowBytes;
-constexpr int kSmem = 4 * kTileBytes + 2 * kTile * 4 + 2 * 128 * 4 + 16 + 128;
+constexpr int kRowMapBytes = 2 * kTile * 4;    // [2][kTile] key row of each slot
+constexpr int kMergeBytes = 2 * 128 * 4;       // a cluster's per-head (max, sum) partials
+constexpr int kMaskBytes = 16;                 // [2][2] slot-validity bits
+constexpr int kSmem = 4 * kTileBytes + kRowMapBytes + kMergeBytes + kMaskBytes + 128;
 constexpr int kMaxSplit = 8;             // CTAs (one cluster) sharing a row's keys
 
 struct SfaArgs {
@@ -152,7 +158,7 @@ __global__ void __launch_bounds__(32 * NW) sfa_kernel(const SfaArgs a)
     uint8_t *sK = base;                                      // [2] key tiles
     uint8_t *sV = base + 2 * kTileBytes;                     // [2] value tiles
     int32_t *sRow = reinterpret_cast<int32_t *>(base + 4 * kTileBytes);   // [2][kTile] key row, -1 = none
-    uint32_t *sMask = reinterpret_cast<uint32_t *>(base + 4 * kTileBytes + 2 * kTile * 4 + 2 * 128 * 4);   // [2][2]
+    uint32_t *sMask = reinterpret_cast<uint32_t *>(base + 4 * kTileBytes + kRowMapBytes + kMergeBytes);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, c = lane & 3;
@@ -364,7 +370,7 @@ __global__ void __launch_bounds__(32 * NW) sfa_kernel(const SfaArgs a)
     if constexpr (C > 1) {
         // partials into this CTA's shared memory (the tile buffers are free)
         float *sO = reinterpret_cast<float *>(base);                 // [N1][128], unnormalised
-        float *sM = reinterpret_cast<float *>(base + 4 * kTileBytes + 2 * kTile * 4);   // [N1]
+        float *sM = reinterpret_cast<float *>(base + 4 * kTileBytes + kRowMapBytes);    // [N1]
         float *sL = sM + 128;                                        // [N1]
         const int h0 = warp * 16 + g, h1 = h0 + 8;
 #pragma unroll

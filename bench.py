@@ -321,9 +321,13 @@ def blas_threads():
         return 1
 
 
-def sfa_workload(name):
+def sfa_workload(name, rank=0):
+    """The named sparse attention workload; rank r > 0 draws an independent
+    problem of the same shape (seed offset by r)."""
     from synth import sfa as ssfa
-    return ssfa.make_sfa_prefill() if name == "sfa_prefill" else ssfa.make_sfa_decode()
+    if name == "sfa_prefill":
+        return ssfa.make_sfa_prefill(seed=9 + rank)
+    return ssfa.make_sfa_decode(seed=10 + rank)
 
 
 def sfa_counts(p, inp):
@@ -384,7 +388,7 @@ def sfa_main(args, ws, rank, local):
         libbuild.build()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    p, inp = sfa_workload(args.workload)
+    p, inp = sfa_workload(args.workload, rank)
     pairs, flops, gathered, io = sfa_counts(p, inp)
     d = {k: v.to(dev) for k, v in inp.items()}
     pr = li.make_sfa_params(p)

@@ -70,3 +70,16 @@ def test_reference_arm_other_ranks_exit_without_work(capsys):
 def test_single_process_reduction_is_identity():
     assert bench.allreduce_max(4.25, device="cpu") == 4.25
     assert not torch.distributed.is_initialized()
+
+
+def test_sfa_reference_arm_other_ranks_exit_without_work(capsys):
+    args = argparse.Namespace(workload="sfa_decode", steps=1, warmup=3)
+    assert bench.sfa_reference(args, 1) == 0
+    assert capsys.readouterr().out == ""
+
+
+def test_sfa_ranks_draw_independent_problems():
+    p0, x0 = bench.sfa_workload("sfa_decode", 0)
+    p1, x1 = bench.sfa_workload("sfa_decode", 1)
+    assert p0.N1 == p1.N1 and p0.sparse_count == p1.sparse_count and p0.rows == p1.rows
+    assert not torch.equal(x0["query"], x1["query"])

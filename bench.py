@@ -423,12 +423,14 @@ def sfa_main(args, ws, rank, local):
     barrier()
     torch.cuda.synchronize()
     launches = 0
+    torch.cuda.nvtx.range_push("timed steps")
     for s_ in range(K):
         flush_l2()
         st_ev[s_].record()
         call()
         en_ev[s_].record()
         launches += li.li_last_launch_count()
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     barrier()
     own = sum(st_ev[s_].elapsed_time(en_ev[s_]) for s_ in range(K))
@@ -598,14 +600,18 @@ def main():
         barrier()
         torch.cuda.synchronize()
         nlaunch = 0
+        torch.cuda.nvtx.range_push("timed steps%s" % (" (stage events)" if stage_events else ""))
         for s in range(K):
             flush_l2()
             if stage_events:
                 li.li_set_profile_events(prof[s])
+            torch.cuda.nvtx.range_push("step %d" % s)
             starts[s].record()
             call(*args_dev)
             ends[s].record()
+            torch.cuda.nvtx.range_pop()
             nlaunch += li.li_last_launch_count()
+        torch.cuda.nvtx.range_pop()
         li.li_set_profile_events(None)
         torch.cuda.synchronize()
         barrier()

@@ -71,6 +71,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a)
     __shared__ int32_t s_ustart[kSmemBlocks];     // unit_start of block g
     const bool in_smem = a.B <= kSmemBatches;
     const int tid = threadIdx.x;
+    // let the score kernel's CTAs launch and run their prologue now; its
+    // griddepcontrol.wait still waits for this grid's completion and writes
+    grid_launch_dependents();
     if (tid == 0) s_flags = 0;
     __syncthreads();
 

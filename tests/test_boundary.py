@@ -206,6 +206,14 @@ def test_oracle_and_cuda_path_share_no_source():
         assert "oracle" not in txt.lower(), f
     pkg = open(os.path.join(ROOT, "sparse_attention_top_n1_b200", "__init__.py")).read()
     assert "import oracle" not in pkg and "from oracle" not in pkg
+    for f in ("sfa.py", "__init__.py"):
+        src = open(os.path.join(ROOT, "oracle", f)).read()
+        assert "sparse_attention_top_n1_b200" not in src, f
+        assert "csrc" not in src, f
+    for f in os.listdir(os.path.join(ROOT, "synth")):
+        if f.endswith(".py"):
+            src = open(os.path.join(ROOT, "synth", f)).read()
+            assert "import oracle" not in src and "sparse_attention_top_n1_b200" not in src, f
 
 
 # ---------------------------------------------------------------- sparse attention

@@ -449,8 +449,12 @@ __device__ bool bucket_topk(const RowSrc &src, int n, int k, int m, int kmax, co
     __syncthreads();
     if (sh.maxbin > (uint32_t)kBinLimit || cstar > (uint32_t)kCandLimit) return false;
 
-    // scatter: selected buckets into keyA/idxA at their bucket slots, the
-    // threshold bucket into keyB/idxB
+    // scatter: selected buckets into their bucket slots, the threshold bucket
+    // into the candidate list.  Each key travels as one 64-bit word,
+    // (key << 32) | ~index, so that one compare orders by value and, for equal
+    // values, by lower index; the words overlay keyA/idxA and candK/candI.
+    uint64_t *wA = reinterpret_cast<uint64_t *>(s.keyA);
+    uint64_t *wC = reinterpret_cast<uint64_t *>(s.candK);
     for (int j4 = tid; j4 < n4; j4 += kTopkThreads) {
         const uint4 q = src.load4(j4);
         const uint32_t kv[4] = {q.x, q.y, q.z, q.w};
@@ -459,14 +463,13 @@ __device__ bool bucket_topk(const RowSrc &src, int n, int k, int m, int kmax, co
             const int j = j4 * 4 + e;
             if (j >= n) break;
             const int b = bucket_of(kv[e], fmin, scale);
+            const uint64_t word = ((uint64_t)kv[e] << 32) | (uint32_t)~(uint32_t)j;
             if (b > bstar) {
                 const uint32_t pos = atomicAdd(&cur[b], 1u);
-                s.keyA[pos] = kv[e];
-                s.idxA[pos] = j;
+                wA[pos] = word;
             } else if (b == bstar) {
                 const uint32_t pos = atomicAdd(&cur[b], 1u) - above;
-                s.candK[pos] = kv[e];
-                s.candI[pos] = j;
+                wC[pos] = word;
             }
         }
     }
@@ -475,30 +478,23 @@ __device__ bool bucket_topk(const RowSrc &src, int n, int k, int m, int kmax, co
     // the threshold bucket: keep the `need` best, ranked among themselves
     const uint32_t need = (uint32_t)m - above;
     for (uint32_t e = tid; e < cstar; e += kTopkThreads) {
-        const uint32_t kv = s.candK[e];
-        const int32_t iv = s.candI[e];
+        const uint64_t w = wC[e];
         uint32_t r = 0;
-        for (uint32_t q = 0; q < cstar; ++q) {
-            const uint32_t kq = s.candK[q];
-            r += (kq > kv) | ((kq == kv) & (s.candI[q] < iv));
-        }
+        for (uint32_t q = 0; q < cstar; ++q) r += wC[q] > w;
         if (r < need) {
-            oidx[above + r] = iv;
-            if (oval) oval[above + r] = from_key(kv);
+            oidx[above + r] = (int32_t)~(uint32_t)w;
+            if (oval) oval[above + r] = from_key((uint32_t)(w >> 32));
         }
     }
     // the buckets above it: bucket offset + rank inside the bucket
     for (uint32_t p = tid; p < above; p += kTopkThreads) {
-        const uint32_t kv = s.keyA[p];
-        const int32_t iv = s.idxA[p];
+        const uint64_t w = wA[p];
+        const uint32_t kv = (uint32_t)(w >> 32);
         const int b = bucket_of(kv, fmin, scale);
         const uint32_t cnt = hist[b], s0 = cur[b] - cnt;
         uint32_t r = 0;
-        for (uint32_t q = s0; q < s0 + cnt; ++q) {
-            const uint32_t kq = s.keyA[q];
-            r += (kq > kv) | ((kq == kv) & (s.idxA[q] < iv));
-        }
-        oidx[s0 + r] = iv;
+        for (uint32_t q = s0; q < s0 + cnt; ++q) r += wA[q] > w;
+        oidx[s0 + r] = (int32_t)~(uint32_t)w;
         if (oval) oval[s0 + r] = from_key(kv);
     }
     for (int j = m + tid; j < k; j += kTopkThreads) {

@@ -19,10 +19,13 @@
 //              (M = 128 keys, N = queries*heads <= 256, K = D) into one of two
 //              fp32 TMEM accumulators, then commits to the ring / accumulator
 //              barriers.
-//   warps 2-9  epilogue: each thread owns one key (one TMEM lane), loads that
-//              lane's head columns with tcgen05.ld and reduces them in
-//              registers -- ReLU, multiply by the weight, sum over heads, scale
-//              -- then writes the score if the key is visible.
+//   warps 2-17 epilogue, two groups of eight, one per accumulator (group g
+//              takes every other tile): each thread owns one key (one TMEM
+//              lane), streams that lane's head columns out of TMEM 16 at a
+//              time (double-buffered, the accumulator handed back once the
+//              last chunk is in registers) and reduces them in registers --
+//              ReLU, multiply by the weight, sum over heads, scale -- then
+//              writes the score if the key is visible.
 // Work is a flat list of (query block, key tile) units written by the
 // device-side scheduler; each CTA takes a contiguous, equal share, so causal
 // triangles and ragged lengths are balanced over the SMs.

@@ -352,6 +352,7 @@ li_status run(const li_params *pp, bool quant, const void *query, const void *ke
     pa.pa_capacity = (int64_t)p.max_blocks_per_seq * p.block_size;
     pa.cmp_res = cmp_shift > 0 && p.sparse_mode == 3 ? p.cmp_residual_k : nullptr;
     pa.cmp_shift = cmp_shift;
+    pa.q_cost = quant ? kQCost8 : kQCost16;
     if (!prof_mark(0, s)) return fail(LI_ERR_CUDA, "recording profile event 0 failed");
     cudaError_t e = launch_plan(pa, s);
     if (e != cudaSuccess) return fail(LI_ERR_CUDA, "scheduler launch: %s", cudaGetErrorString(e));
@@ -387,6 +388,7 @@ li_status run(const li_params *pp, bool quant, const void *query, const void *ke
     const uint32_t fmt = kind == kKindF16 ? (p.dtype_qk == LI_BF16 ? 1u : 0u) : (kind == kKindI8 ? 1u : 0u);
     sa.idesc_base = make_idesc(fmt, fmt, 128, 0, kind == kKindI8 ? 2u : 1u);
     sa.cmp_shift = cmp_shift;
+    sa.q_cost = pa.q_cost;
     sa.dtype_scale = p.dtype_scale;
     sa.timeout_ns = kDefaultTimeoutNs;
     e = launch_score(sa, t, qmap, kmap, kind, sms, s);

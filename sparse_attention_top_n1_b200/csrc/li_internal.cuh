@@ -16,7 +16,11 @@ constexpr int kAccCols = 256;         // TMEM columns per accumulator (the N axi
 constexpr int kAccStages = 2;         // double-buffered accumulators (512 TMEM columns)
 constexpr int kGroupWarps = 8;        // warps of one epilogue group (2 per TMEM lane quarter)
 constexpr int kEpiWarps = kAccStages * kGroupWarps;   // one group per accumulator
-constexpr int kQCost = 2;             // scheduler weight of one query-tile load, in key tiles
+// Scheduler weight of one query-tile load, in key tiles: the bubble a block
+// switch costs relative to one tile's work.  8-bit keys make a tile cheaper
+// (half the MMA time and bytes), so a block switch weighs more.
+constexpr int kQCost16 = 2;           // bf16 / fp16 q/k
+constexpr int kQCost8 = 4;            // fp8 / int8 q/k
 constexpr int kScoreThreads = 32 * (2 + kEpiWarps);
 constexpr int kTopkThreads = 512;
 constexpr int kPlanThreads = 1024;
@@ -95,6 +99,7 @@ struct PlanArgs {
     int32_t grid;          // score CTAs
     const int32_t *cmp_res;  // [B] residual original key tokens (NULL: none)
     int32_t cmp_shift;       // log2(cmp_ratio)
+    int32_t q_cost;          // weight of a query-tile load (kQCost16 or kQCost8)
 };
 
 struct ScoreArgs {
@@ -115,6 +120,7 @@ struct ScoreArgs {
     int32_t q_single, k_single; // one copy covers both 128-byte chunks (3-D / 4-D maps)
     uint32_t idesc_base;        // instruction descriptor without N
     int32_t cmp_shift;          // log2(cmp_ratio): compressed keys under mode 3
+    int32_t q_cost;             // weight of a query-tile load in the work list
     int64_t timeout_ns;
 };
 

@@ -11,7 +11,7 @@
 //   BatchInfo[b]  clamped lengths and offsets of every batch
 //   BlockInfo[g]  query block g: its batch, first query, the number of key
 //                 tiles its last (most-seeing) query needs, and its first
-//                 position in the weighted work list (tiles + kQCost per block)
+//                 position in the weighted work list (tiles + q_cost per block)
 //   cta_start[c]  where score CTA c's equal share of the work list begins:
 //                 its first block, tile, and that block's unit_start and
 //                 tile count (one load for the CTA instead of a search)
@@ -192,7 +192,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a)
             blk.ntiles = ntiles;
         }
         // a block weighs its key tiles plus the cost of loading its query tile
-        const int32_t weight = ntiles > 0 ? ntiles + kQCost : 0;
+        const int32_t weight = ntiles > 0 ? ntiles + a.q_cost : 0;
         int32_t incl = weight;
         const int32_t tot = block_inclusive_scan(incl, s_tmp);
         if (g < total_blocks) {
@@ -226,9 +226,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a)
             const int32_t u1 = lo + 1 < total_blocks
                                    ? (ustart_in_smem ? s_ustart[lo + 1] : a.blocks[lo + 1].unit_start)
                                    : total_units;
-            int32_t tile = w0 - u0 - kQCost;
+            int32_t tile = w0 - u0 - a.q_cost;
             if (tile < 0) tile = 0;
-            st = make_int4(lo, tile, u0, u1 - u0 - kQCost);
+            st = make_int4(lo, tile, u0, u1 - u0 - a.q_cost);
         }
         a.cta_start[c] = st;
     }

@@ -56,12 +56,12 @@ struct Geometry {
 };
 
 // Walks this CTA's share [w0, w1) of the weighted work list.  A block of n
-// key tiles occupies n + kQCost consecutive positions: kQCost for loading its
+// key tiles occupies n + q_cost consecutive positions: q_cost for loading its
 // query tile, then one per key tile; a tile belongs to the CTA whose range
 // holds its position, so every tile is processed exactly once.
 struct Walker {
     const BlockInfo *blocks;
-    int nblocks, w_end;
+    int nblocks, w_end, qcost;
     int qb, tile, ntiles, start;
     __device__ void load_block()
     {
@@ -89,7 +89,7 @@ struct Walker {
         start = st.z;
         ntiles = st.w;
     }
-    __device__ bool valid() const { return qb < nblocks && start + kQCost + tile < w_end; }
+    __device__ bool valid() const { return qb < nblocks && start + qcost + tile < w_end; }
     __device__ void next()
     {
         ++tile;
@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         // per-tile block lookups are shared-memory reads, not dependent
         // global loads on the copy path.
         if (w_begin < w_end && nblocks > 0) {
-            Walker w{a.blocks, nblocks, 0, 0, 0, 0, 0};
+            Walker w{a.blocks, nblocks, 0, a.q_cost, 0, 0, 0, 0};
             w.init_from(a.cta_start[blockIdx.x], w_end);
             int stage = 0, prev_qb = -1;
             uint32_t phase = 0, qphase = 0;
@@ -440,7 +440,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0 && w_begin < w_end && nblocks > 0) {
-            Walker w{a.blocks, nblocks, 0, 0, 0, 0, 0};
+            Walker w{a.blocks, nblocks, 0, a.q_cost, 0, 0, 0, 0};
             w.init_from(a.cta_start[blockIdx.x], w_end);
             int stage = 0, acc = 0, prev_qb = -1;
             uint32_t phase = 0, acc_phase = 0, qphase = 0, idesc = 0;
@@ -520,7 +520,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         const int lrow = quarter * 32 + lane;      // key row within the tile
         float *myW = sW + ew * 128;
         if (w_begin < w_end && nblocks > 0) {
-            Walker w{a.blocks, nblocks, 0, 0, 0, 0, 0};
+            Walker w{a.blocks, nblocks, 0, a.q_cost, 0, 0, 0, 0};
             w.init_from(a.cta_start[blockIdx.x], w_end);
             const int acc = grp;
             int prev_qb = -1, nchunks = 0, parity = 0;

@@ -1,11 +1,13 @@
 """Python binding of libli, the B200 LightningIndexer (C ABI in include/li.h).
 
-The binding only marshals arguments: every step of the indexer runs in the
-CUDA kernels of ``libli.so``.  Functions keep the C names (``li_indexer``,
-``li_quant_indexer``, ``li_topk``, ``li_output_shape``, ``li_workspace_size``,
-``li_read_device_status``, ...) and take torch CUDA tensors, passing their
-device pointers and the current CUDA stream.  ``indexer(...)`` is a
-convenience wrapper that allocates the outputs and workspace with torch.
+The binding only marshals arguments: every step of the indexer and of the
+sparse attention that consumes its output runs in the CUDA kernels of
+``libli.so``.  Functions keep the C names (``li_indexer``,
+``li_quant_indexer``, ``li_topk``, ``li_sparse_attention``,
+``li_output_shape``, ``li_workspace_size``, ``li_read_device_status``, ...)
+and take torch CUDA tensors, passing their device pointers and the current
+CUDA stream.  ``indexer(...)`` and ``sparse_attention(...)`` are convenience
+wrappers that allocate the outputs (and the indexer's workspace) with torch.
 
 There is no fallback: if ``libli.so`` is missing or fails to load, importing
 the functions raises.

@@ -170,9 +170,28 @@ def pin_empty_rows(mut):
     return bool(ok)
 
 
+def pin_split_merge(mut):
+    """Attention over a key set equals the merge of attention over any split of
+    it: with (out_s, lse_s) per part, LSE = logsumexp_s lse_s and
+    out = sum_s exp(lse_s - LSE) * out_s (the rule split rows are merged by)."""
+    p, x = ssfa.make_sfa(21, B=1, S1=3, S2=200, N1=16, K=96, causal=False)
+    full = osfa.run(p, x, rows=[1], mutation=mut)
+    row = x["sparse_indices"][1, 0].tolist()
+    parts = [row[:17], row[17:60], row[60:]]
+    outs, lses = [], []
+    for part in parts:
+        r = osfa.run(p, _set_row(x, 1, part), rows=[1], mutation=mut)
+        outs.append(r["out"][0])
+        lses.append(r["lse"][0])
+    L = np.logaddexp.reduce(np.stack(lses), axis=0)                  # [N1]
+    merged = sum(np.exp(l - L)[:, None] * o for l, o in zip(lses, outs))
+    return bool(np.allclose(merged, full["out"][0], rtol=1e-12, atol=1e-12)
+                and np.allclose(L, full["lse"][0], rtol=1e-12, atol=1e-12))
+
+
 PINS = [pin_single_key, pin_zero_query_mean, pin_order_invariance, pin_library_sdpa,
         pin_huge_gap_argmax, pin_skips_invalid, pin_layout_invariance, pin_scale_fold,
-        pin_empty_rows]
+        pin_empty_rows, pin_split_merge]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[f.__name__ for f in PINS])

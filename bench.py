@@ -4,23 +4,35 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 One step is one full indexer call (all three kernels) over one batch of the
-named synthetic workload, with inputs resident in HBM.  The ``sfa_*``
-workloads instead time one call of the sparse attention consumer
-(li_sparse_attention) over its own synthetic inputs.  The default workload
-is the TileLang test shape (B=2, S1=512, S2=4096, G=32, D=64, k=1024, fp16,
-no mask).  L2 is flushed before every timed step (a 256 MiB device write,
-then a 256 MiB read of a second buffer so no dirty lines are left behind),
-outside the timed interval; each step is timed with CUDA events on the
-launching stream and the per-step times are summed.  Under torchrun every
-rank runs its own copy of the workload (independent problems, weak scaling,
-no data-path collective); the job time is the max over ranks.
+named synthetic workload, with inputs resident in HBM.  The default workload
+is the largest of the five configurations: the quantised varlen prefill (TND,
+sequences of 2048/4096/8192/16384 tokens, 64 heads, D = 128, fp8 e4m3 q/k
+with fp32 dequant scales, k = 2048, right-down causal).  With one GPU the
+same run also times the other four configurations (tiny, the TileLang test
+shape, DSA prefill and paged decode) and reports each under ``per_config``,
+with its stage times, roofline, clocks and oracle baseline.
 
-The JSON line reports queries/s (value), the effective TFLOP/s, the roofline
-of the dominant kernel measured live with per-stage CUDA events, an
-end-to-end figure through the C ABI with host buffers (copies inside the
-timed region), and the fp64 oracle timed on the host cores on a bounded
-sample (cpu_baseline).  `--impl reference` times that oracle alone as the
-reference arm.
+L2 is flushed before every timed step (a 256 MiB device write, then a
+256 MiB read of a second buffer so no dirty lines are left behind), outside
+the timed interval; each step is timed with CUDA events on the launching
+stream and the per-step times are summed.
+
+Under torchrun (N > 1) the problem is split by query rows: each rank takes a
+contiguous row range balanced by visible pairs, keeps its own copy of the
+keys and runs its rows through the ordinary entry points (one to three calls
+per step).  Nothing crosses ranks on the data path; the job time is the max
+over ranks and the value is the problem's rows over that time (strong
+scaling).
+
+The JSON line reports queries/s (value), the effective TFLOP/s, per-kernel
+rooflines measured live with per-stage CUDA events (each kernel's bound is
+the slower of its FLOPs at the tensor peak of its operand type and its bytes
+at the HBM peak), an end-to-end figure through the C ABI with host buffers
+(copies inside the timed region), and the fp64 oracle timed on the host cores
+on a bounded sample (cpu_baseline).  The fp8 and int8 dense tensor peaks are
+measured in the same run (cuBLAS through torch, 8192^3, best of 10), since
+the driver's peak file holds only bf16.  `--impl reference` times the oracle
+alone as the reference arm.
 """
 from __future__ import annotations
 
@@ -39,7 +51,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "indexer queries/s and effective TFLOP/s at 1 B200; % of tensor/HBM roofline"
 UNIT = "queries/s"
-DEFAULT_WORKLOAD = "cfg2"
+DEFAULT_WORKLOAD = "quant_varlen"
+# the five configurations of the benchmark, timed together when N = 1
+CONFIGS = ("tiny", "cfg2", "dsa_prefill", "paged_decode", "quant_varlen")
 FLUSH_BYTES = 256 << 20
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -56,36 +70,33 @@ WORKLOAD_DESC = {
     "sfa_prefill": "sparse attention consumer of DSA prefill: 8192 rows x 64 heads, K=2048 selected keys (causal), D=Dv=128 bf16",
     "sfa_decode": "sparse attention consumer of paged decode: 64 rows x 64 heads over a PA pool (block 128, lengths U[4096,65536]), K=2048, D=Dv=128 bf16",
 }
-SFA_METRIC = "sparse attention query rows/s at 1 B200 (the indexer's consumer); % of tensor roofline"
+SFA_METRIC = "sparse attention query rows/s at 1 B200 (the indexer's consumer); % of tensor/HBM roofline"
 SFA_UNIT = "rows/s"
 RETURN_VALUE = {"tiny": 1, "cfg2": 1, "dsa_prefill": 1, "paged_decode": 0, "quant_varlen": 0,
                 "quant_varlen_int8": 0, "quant_int8_pa": 0, "dsa_prefill_window": 1}
-
-
 SEEDS = {"tiny": 0, "cfg2": 1, "dsa_prefill": 2, "paged_decode": 3, "quant_varlen": 4,
          "quant_int8_pa": 5, "quant_varlen_int8": 6, "dsa_prefill_window": 7}
+DTYPE_NAME = {"bf16": "bf16", "fp16": "fp16", "e4m3": "fp8_e4m3", "int8": "int8"}
 
 
-def make_workload(name, rank=0):
-    """The named workload; rank r > 0 draws an independent problem of the same
-    shape (seed offset by r), as weak scaling over independent problems."""
+def make_workload(name, seed_offset=0):
+    """The named workload (seed offset only for tests of independent draws)."""
     import synth
     fn = synth.WORKLOADS[name]
     if name in ("tiny",):
-        return fn(seed=SEEDS[name] + rank)
-    return fn(seed=SEEDS[name] + rank, return_value=RETURN_VALUE[name])
+        return fn(seed=SEEDS[name] + seed_offset)
+    return fn(seed=SEEDS[name] + seed_offset, return_value=RETURN_VALUE[name])
 
 
-def job_value(rows_per_rank, steps, world, max_total_ms):
-    """Whole-job queries/s: every rank's rows over the slowest rank's time."""
-    return world * rows_per_rank * steps / (max_total_ms * 1e-3)
+def job_value(rows, steps, max_total_ms):
+    """Whole-job queries/s: the problem's rows per step over the slowest rank's time."""
+    return rows * steps / (max_total_ms * 1e-3)
 
 
-def work_counts(p, inp):
-    """Host-side algorithmic work: visible pairs, FLOPs and compulsory bytes."""
-    import torch
-    B = p.B
+def seq_lengths(p, inp):
+    """Per-batch query and key lengths (host lists)."""
     aq, ak = inp.get("act_q"), inp.get("act_k")
+    B = p.B
     if p.layout_q == "TND":
         cq = [0] + aq.tolist()
         Sq = [cq[b + 1] - cq[b] for b in range(B)]
@@ -98,37 +109,125 @@ def work_counts(p, inp):
         Sk = ak.tolist() if ak is not None else [p.S2] * B
     else:
         Sk = ak.tolist()
+    return Sq, Sk
+
+
+def work_counts(p, inp):
+    """Host-side algorithmic work of one call: visible pairs, FLOPs, and the
+    bytes each kernel must move at least.
+
+    * score kernel: its inputs (query, each key once, weights, scales, block
+      table, lengths) plus one fp32 score per visible pair written;
+    * Top-k kernel: one fp32 score per visible pair read plus the outputs;
+    * whole call: the inputs plus the outputs (the score rows are an
+      intermediate and do not count).
+    """
+    Sq, Sk = seq_lengths(p, inp)
     pairs = 0
-    rows_nvis = 0
-    for b in range(B):
+    for b in range(p.B):
         if p.sparse_mode == 0:
             pairs += Sq[b] * Sk[b]
         else:
             for i in range(Sq[b]):
                 pairs += max(0, min(Sk[b], i + 1 + Sk[b] - Sq[b]))
-    rows_nvis = pairs
     es = 1 if p.dtype_qk in ("e4m3", "int8") else 2
-    esw = 4 if p.dtype_w == "fp32" else 2
     nbytes = lambda t: 0 if t is None else t.numel() * t.element_size()
-    keys_visible = sum(Sk)
-    kv_bytes = keys_visible * p.D * es
-    compulsory = (nbytes(inp["query"]) + kv_bytes + nbytes(inp["weights"])
-                  + nbytes(inp.get("q_scale"))
-                  + keys_visible * (4 if p.dtype_scale == "fp32" else 2) * int(p.quant)
-                  + nbytes(inp.get("block_table")) + nbytes(aq) + nbytes(ak)
-                  + p.rows * p.sparse_count * (4 + 4 * p.return_value))
-    topk_bytes = rows_nvis * 4 + p.rows * p.sparse_count * (4 + 4 * p.return_value)
-    return dict(pairs=pairs, flops=2.0 * p.N1 * p.D * pairs, compulsory_bytes=compulsory,
-                topk_bytes=topk_bytes, score_bytes=compulsory - p.rows * p.sparse_count *
-                (4 + 4 * p.return_value) + pairs * 4, es=es, esw=esw)
+    keys = sum(Sk)
+    inputs = (nbytes(inp["query"]) + keys * p.D * es + nbytes(inp["weights"])
+              + nbytes(inp.get("q_scale"))
+              + keys * (4 if p.dtype_scale == "fp32" else 2) * int(p.quant)
+              + nbytes(inp.get("block_table")) + nbytes(inp.get("act_q")) + nbytes(inp.get("act_k")))
+    outputs = p.rows * p.sparse_count * (4 + 4 * p.return_value)
+    return dict(pairs=pairs, flops=2.0 * p.N1 * p.D * pairs, compulsory_bytes=inputs + outputs,
+                score_bytes=inputs + pairs * 4, topk_bytes=pairs * 4 + outputs, es=es)
 
 
 def load_peaks():
     if os.path.exists(PEAKS_FILE):
         with open(PEAKS_FILE) as f:
             d = json.load(f)
-        return d, "measured"
-    return FALLBACK_PEAKS, "fallback"
+        return d, "measured (MEASURED_PEAKS.json)"
+    print("bench: MEASURED_PEAKS.json is absent; rooflines use the fallback peaks "
+          "(6650 GB/s, 1590 TFLOP/s bf16) and say so", file=sys.stderr)
+    return FALLBACK_PEAKS, "fallback (MEASURED_PEAKS.json absent)"
+
+
+def measure_8bit_peaks(dev, n=8192, reps=10):
+    """Dense fp8 e4m3 and int8 tensor throughput of this GPU through cuBLAS
+    (torch._scaled_mm / torch._int_mm), n^3 GEMMs, best of `reps` after 3
+    warm-up calls, CUDA events.  A figure below the bf16 peak is not trusted
+    (that library path is not on the 8-bit tensor cores) and left None."""
+    import torch
+    out = {"how": "torch._scaled_mm e4m3 (bf16 out) and torch._int_mm int8, %d^3, best of %d, CUDA events"
+           % (n, reps)}
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+
+    def best(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return 2.0 * n ** 3 / (min(ts) * 1e-3) / 1e12
+
+    try:
+        a = torch.randn(n, n, device=dev, generator=g).to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device=dev, generator=g).to(torch.float8_e4m3fn).t()
+        one = torch.ones((), device=dev, dtype=torch.float32)
+        out["fp8_tflops"] = best(lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one,
+                                                          out_dtype=torch.bfloat16))
+        del a, b
+    except Exception as e:  # pragma: no cover - depends on the torch build
+        out["fp8_tflops"] = None
+        out["fp8_error"] = str(e)[:120]
+    try:
+        a = torch.randint(-64, 64, (n, n), device=dev, dtype=torch.int8, generator=g)
+        b = torch.randint(-64, 64, (n, n), device=dev, dtype=torch.int8, generator=g)
+        out["int8_tops"] = best(lambda: torch._int_mm(a, b))
+        del a, b
+    except Exception as e:  # pragma: no cover
+        out["int8_tops"] = None
+        out["int8_error"] = str(e)[:120]
+    torch.cuda.empty_cache()
+    return out
+
+
+def tensor_peak(dtype_qk, peaks, peak_src, p8):
+    """(peak TFLOP/s, description) of the score MMA's operand type."""
+    bf16 = peaks["bf16_tflops"]
+    if dtype_qk in ("bf16", "fp16"):
+        return bf16, "bf16 dense burst peak (fp16 has the same rate), %s" % peak_src
+    key = "fp8_tflops" if dtype_qk == "e4m3" else "int8_tops"
+    v = (p8 or {}).get(key)
+    if v and v >= bf16:
+        return v, "%s dense peak measured in this run (%s)" % ("fp8" if dtype_qk == "e4m3" else "int8", p8["how"])
+    return 2.0 * bf16, "assumed: 2x the bf16 peak (nominal 8-bit/16-bit ratio; the in-run measurement failed)"
+
+
+def roofline(ms, flops, nbytes, t_peak, t_src, hbm, hbm_src, traffic=None):
+    """Bound = the slower of flops at the tensor peak and bytes at HBM bandwidth."""
+    t_t = flops / (t_peak * 1e12) if flops else 0.0
+    t_b = nbytes / (hbm * 1e9)
+    sec = ms * 1e-3
+    if t_t >= t_b:
+        r = {"bound": "tensor", "achieved": flops / sec / 1e12, "peak": t_peak, "unit": "TFLOP/s",
+             "peak_source": t_src}
+    else:
+        r = {"bound": "hbm", "achieved": nbytes / sec / 1e9, "peak": hbm, "unit": "GB/s",
+             "peak_source": "HBM copy peak, %s" % hbm_src}
+    r["frac"] = max(t_t, t_b) / sec
+    r["ms"] = ms
+    r["algorithmic_bytes"] = nbytes
+    r["flops"] = flops
+    r["traffic"] = traffic
+    return r
 
 
 def traffic_record(workload, kernel):
@@ -243,7 +342,7 @@ def cpu_model():
     return platform.processor() or "unknown"
 
 
-def cpu_oracle_sample(p, inp, budget_s=12.0, max_rows=None, seed=0):
+def cpu_oracle_sample(p, inp, budget_s=12.0, seed=0):
     """Time the fp64 oracle on a bounded sample of query rows (host cores)."""
     import numpy as np
 
@@ -255,9 +354,8 @@ def cpu_oracle_sample(p, inp, budget_s=12.0, max_rows=None, seed=0):
     probe = sorted(rng.choice(R, size=min(R, max(nthreads, 8)), replace=False).tolist())
     t0 = time.perf_counter()
     oracle.run(p, inp, rows=probe, nthreads=nthreads)
-    t_probe = time.perf_counter() - t0
-    per_row = t_probe / len(probe)
-    n = int(min(R if max_rows is None else max_rows, max(len(probe), budget_s / max(per_row, 1e-9))))
+    per_row = (time.perf_counter() - t0) / len(probe)
+    n = int(min(R, max(len(probe), budget_s / max(per_row, 1e-9))))
     rows = sorted(rng.choice(R, size=n, replace=False).tolist())
     t0 = time.perf_counter()
     oracle.run(p, inp, rows=rows, nthreads=nthreads)
@@ -265,7 +363,7 @@ def cpu_oracle_sample(p, inp, budget_s=12.0, max_rows=None, seed=0):
     return {"value": len(rows) / dt, "unit": UNIT, "cores": nthreads, "kind": "oracle",
             "cpu_model": cpu_model(), "nproc": os.cpu_count(),
             "sample": "%d of %d query rows (seeded uniform sample), fp64 C oracle, %.2f s"
-                      % (len(rows), R, dt)}, rows, dt
+                      % (len(rows), R, dt)}
 
 
 def run_reference(args, ws, rank):
@@ -299,7 +397,7 @@ def run_reference(args, ws, rank):
     value = n * len(times) / tot
     line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
             "config": {"workload": WORKLOAD_DESC[args.workload], "rows_per_step": n},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle",
@@ -321,23 +419,282 @@ def blas_threads():
         return 1
 
 
-def sfa_workload(name, rank=0):
-    """The named sparse attention workload; rank r > 0 draws an independent
-    problem of the same shape (seed offset by r)."""
+# ------------------------------------------------------------------ indexer
+
+def make_flush(dev):
+    import torch
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    clean = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)   # fp32: summed without a cast
+
+    def flush_l2():
+        """Evict L2: write a buffer larger than L2, then read a second one, so
+        that the written lines are back in HBM before the next step starts and
+        the timed step does not inherit their write-back."""
+        flush.zero_()
+        clean.sum()
+    return flush_l2
+
+
+class Calls:
+    """This rank's calls of one step: the whole problem at N = 1, else the
+    pieces of its row range (sparse_attention_top_n1_b200.shard)."""
+
+    def __init__(self, li, p, inp, dev, ws, rank):
+        import dataclasses
+
+        import torch
+
+        from sparse_attention_top_n1_b200 import shard
+        self.li = li
+        self.p = p
+        self.quant = bool(p.quant)
+        shape = (p.rows, p.sparse_count)
+        self.idx = torch.empty(shape, dtype=torch.int32, device=dev)
+        self.val = torch.empty(shape, dtype=torch.float32, device=dev) if p.return_value else None
+        self.d = {k: v.to(dev) for k, v in inp.items()}
+        self.host_inputs = inp
+        if ws == 1:
+            self.pieces = [(p, self.d, 0, p.rows, inp)]
+        else:
+            plan = shard.shard(p, ws, inp.get("act_q"), inp.get("act_k"), inp.get("cmp_residual_k"))[rank]
+            to_dev = lambda a: torch.from_numpy(a).to(dev)
+            self.pieces = [(dataclasses.replace(p, **pc.fields), shard.piece_inputs(pc, p, self.d, to_dev),
+                            pc.r0, pc.r1, shard.piece_inputs(pc, p, inp)) for pc in plan]
+        self.calls = []
+        for sp, sd, r0, r1, _ in self.pieces:
+            pr = li.make_params(sp)
+            if sd.get("cmp_residual_k") is not None:
+                pr.cmp_residual_k = sd["cmp_residual_k"].data_ptr()
+            wsb = li.alloc_workspace(pr, dev)
+            oi = self.idx[r0:r1]
+            ov = self.val[r0:r1] if self.val is not None else None
+            self.calls.append((pr, sd, wsb, oi, ov))
+        self.rows_here = sum(r1 - r0 for _, _, r0, r1, _ in self.pieces)
+
+    def __call__(self, prof=None):
+        li = self.li
+        n = 0
+        for j, (pr, sd, wsb, oi, ov) in enumerate(self.calls):
+            if prof is not None:
+                li.li_set_profile_events(prof[j])
+            if self.quant:
+                li.li_quant_indexer(pr, sd["query"], sd["key"], sd["weights"], sd.get("q_scale"),
+                                    sd.get("k_scale"), sd.get("act_q"), sd.get("act_k"),
+                                    sd.get("block_table"), oi, ov, wsb)
+            else:
+                li.li_indexer(pr, sd["query"], sd["key"], sd["weights"], sd.get("act_q"),
+                              sd.get("act_k"), sd.get("block_table"), oi, ov, wsb)
+            n += li.li_last_launch_count()
+        if prof is not None:
+            li.li_set_profile_events(None)
+        return n
+
+    def device_flags(self):
+        f = 0
+        for _, _, wsb, _, _ in self.calls:
+            f |= self.li.li_read_device_status(wsb)
+        return f
+
+
+def time_indexer(name, args, ctx, steps, warmup, cpu_budget, with_e2e=True):
+    """Time `steps` calls of workload `name` on this rank; returns the record."""
+    import torch
+    li, dev, ws, rank = ctx["li"], ctx["dev"], ctx["ws"], ctx["rank"]
+    p, inp = make_workload(name)
+    counts = work_counts(p, inp)
+    calls = Calls(li, p, inp, dev, ws, rank)
+    flush_l2 = ctx["flush"]
+    clocks = ClockSampler(ctx["local"])
+    if not args.plain:
+        clocks.start()
+    # W warm-up steps, then more of the same until the clock sampler has seen
+    # the GPU under this load for a while (its period is 200 ms)
+    t_warm = time.perf_counter()
+    nwarm = 0
+    while nwarm < warmup or (not args.plain and time.perf_counter() - t_warm < 0.8):
+        flush_l2()
+        calls()
+        nwarm += 1
+        if nwarm % 16 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
+    flags = calls.device_flags()
+    if flags:
+        raise SystemExit("%s: device status 0x%x during warm-up" % (name, flags))
+
+    K = steps
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    ncalls = len(calls.calls)
+
+    def timed_steps(stage_events):
+        """K steps, L2 flushed before each outside the timed interval.  With
+        stage_events, the library records per-kernel events inside each call
+        (which keeps the kernels from overlapping their launch with the
+        previous kernel's tail, so the step itself gets a little slower)."""
+        starts = [mk() for _ in range(K)]
+        ends = [mk() for _ in range(K)]
+        prof = [[[mk() for _ in range(4)] for _ in range(ncalls)] for _ in range(K)]
+        for e in [x for st in prof for c in st for x in c]:      # torch creates events lazily
+            e.record()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        nlaunch = 0
+        torch.cuda.nvtx.range_push("timed steps%s" % (" (stage events)" if stage_events else ""))
+        for s in range(K):
+            flush_l2()
+            torch.cuda.nvtx.range_push("step %d" % s)
+            starts[s].record()
+            nlaunch += calls(prof[s] if stage_events else None)
+            ends[s].record()
+            torch.cuda.nvtx.range_pop()
+        torch.cuda.nvtx.range_pop()
+        torch.cuda.synchronize()
+        barrier()
+        step_ms = [starts[s].elapsed_time(ends[s]) for s in range(K)]
+        stage = {"scheduler": [], "score": [], "topk": []}
+        if stage_events:
+            for s in range(K):
+                sch = sc = tk = 0.0
+                for e in prof[s]:
+                    sch += e[0].elapsed_time(e[1])
+                    sc += e[1].elapsed_time(e[2])
+                    tk += e[2].elapsed_time(e[3])
+                stage["scheduler"].append(sch)
+                stage["score"].append(sc)
+                stage["topk"].append(tk)
+        return sum(step_ms), stage, nlaunch
+
+    # timed region 1: the job value, nothing between the kernels
+    own_ms, _, launches = timed_steps(False)
+    total_ms = allreduce_max(own_ms)
+    # timed region 2: the same steps with per-kernel events, for the roofline
+    staged_ms = 0.0
+    stage = {"scheduler": [], "score": [], "topk": []}
+    if not args.no_stage_events:
+        own_staged, stage, _ = timed_steps(True)
+        staged_ms = allreduce_max(own_staged)
+    clk = clocks.stop()
+    avg = {k: (sum(v) / len(v) if v else float("nan")) for k, v in stage.items()}
+    # the slowest rank's stage times (the roofline of the job)
+    avg = {k: allreduce_max(v) for k, v in avg.items()}
+
+    peaks, peak_src, p8 = ctx["peaks"], ctx["peak_src"], ctx["p8"]
+    tpk, tsrc = tensor_peak(p.dtype_qk, peaks, peak_src, p8)
+    hbm = peaks["hbm_gbs"]
+    share = 1.0 / ws            # each rank does about 1/N of the pairs and rows
+    kern = {}
+    if avg["score"] == avg["score"]:          # not NaN
+        kern["score"] = roofline(avg["score"], counts["flops"] * share,
+                                 counts["score_bytes"] * share, tpk, tsrc, hbm, peak_src,
+                                 traffic_record(name, "score") if ws == 1 else None)
+        kern["topk"] = roofline(avg["topk"], 0.0, counts["topk_bytes"] * share, tpk, tsrc, hbm,
+                                peak_src, traffic_record(name, "topk") if ws == 1 else None)
+    ms_step = total_ms / K
+    whole = roofline(ms_step, counts["flops"], counts["compulsory_bytes"], tpk * ws, tsrc,
+                     hbm * ws, peak_src)
+    dom = max(kern, key=lambda k: kern[k]["ms"]) if kern else None
+    roof = None
+    if dom:
+        roof = {k: kern[dom][k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic",
+                                          "peak_source")}
+        roof["kernel"] = dom + "_kernel"
+
+    # end to end through the C ABI with host buffers: H2D of this rank's inputs
+    # from pinned memory, the call, D2H of its output rows, all timed
+    e2e = None
+    if with_e2e and not (args.no_e2e or args.plain):
+        # every device tensor a call reads is refreshed once per step (pieces
+        # that share one, such as a paged pool, copy it once)
+        hosts = []
+        h2d = 0
+        seen = set()
+        for (sp, sd, r0, r1, hin), (pr, dd, wsb, oi, ov) in zip(calls.pieces, calls.calls):
+            hp = {}
+            for k, v in hin.items():
+                if k not in dd or (dd[k].data_ptr(), dd[k].numel()) in seen:
+                    continue
+                seen.add((dd[k].data_ptr(), dd[k].numel()))
+                hp[k] = v.contiguous().pin_memory()
+            h2d += sum(v.numel() * v.element_size() for v in hp.values())
+            hosts.append((hp, dd))
+        hidx = torch.empty(calls.idx.shape, dtype=torch.int32).pin_memory()
+        hval = torch.empty(calls.idx.shape, dtype=torch.float32).pin_memory() if p.return_value else None
+        d2h = calls.rows_here * p.sparse_count * (4 + 4 * p.return_value)
+        e_st = [mk() for _ in range(K + warmup)]
+        e_en = [mk() for _ in range(K + warmup)]
+        for s in range(K + warmup):
+            flush_l2()
+            e_st[s].record()
+            for hp, dd in hosts:
+                for k2, v in hp.items():
+                    dd[k2].copy_(v, non_blocking=True)
+            calls()
+            for _, _, r0, r1, _ in calls.pieces:
+                hidx[r0:r1].copy_(calls.idx[r0:r1], non_blocking=True)
+                if hval is not None:
+                    hval[r0:r1].copy_(calls.val[r0:r1], non_blocking=True)
+            e_en[s].record()
+        torch.cuda.synchronize()
+        e_ms = allreduce_max(sum(e_st[s].elapsed_time(e_en[s]) for s in range(warmup, K + warmup)))
+        e2e = {"value": p.rows * K / (e_ms * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    flags = calls.device_flags()
+    if flags:
+        raise SystemExit("%s: device status 0x%x after timing" % (name, flags))
+
+    cpu = None
+    if rank == 0 and ws == 1 and cpu_budget > 0 and not (args.no_cpu_baseline or args.plain):
+        cpu = cpu_oracle_sample(p, inp, budget_s=cpu_budget)
+
+    rec = {
+        "workload": name, "config": WORKLOAD_DESC[name], "dtype": DTYPE_NAME[p.dtype_qk],
+        "rows": p.rows, "visible_pairs": counts["pairs"], "sparse_count": p.sparse_count,
+        "return_value": p.return_value, "steps": K, "warmup": warmup,
+        "ms_per_step": ms_step, "value": job_value(p.rows, K, total_ms), "unit": UNIT,
+        "ms_per_step_with_stage_events": (staged_ms / K) if staged_ms else None,
+        "effective_tflops": counts["flops"] * K / (total_ms * 1e-3) / 1e12,
+        "whole_call_roofline": {k: whole[k] for k in ("bound", "achieved", "peak", "unit", "frac")},
+        "roofline": roof, "kernels": kern, "stage_ms": avg,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
+        "calls_per_step_this_rank": len(calls.calls),
+    }
+    del calls
+    torch.cuda.empty_cache()
+    return rec
+
+
+# ------------------------------------------------------------------ sparse attention
+
+def sfa_workload(name, seed_offset=0):
     from synth import sfa as ssfa
     if name == "sfa_prefill":
-        return ssfa.make_sfa_prefill(seed=9 + rank)
-    return ssfa.make_sfa_decode(seed=10 + rank)
+        return ssfa.make_sfa_prefill(seed=9 + seed_offset)
+    return ssfa.make_sfa_decode(seed=10 + seed_offset)
 
 
 def sfa_counts(p, inp):
-    """Valid (row, selected key) pairs, FLOPs and gathered bytes of one call."""
-    idx = inp["sparse_indices"].reshape(p.rows, p.sparse_count)
-    pairs = int((idx >= 0).sum())
+    """Valid (row, selected key) pairs, FLOPs, gathered bytes and the bytes one
+    call must move at least (query, output, lse, index rows, and each distinct
+    selected key/value row once)."""
+    import numpy as np
+    idx = inp["sparse_indices"].reshape(p.rows, p.sparse_count).numpy()
+    valid = idx >= 0
+    pairs = int(valid.sum())
     flops = 2.0 * p.N1 * (p.D + p.Dv) * pairs
     gathered = pairs * (p.D + p.Dv) * 2
-    io = p.rows * p.N1 * (p.D + p.Dv) * 2 + idx.numel() * 4 + p.rows * p.N1 * 4
-    return pairs, flops, gathered, io
+    # distinct selected keys per batch
+    if p.layout_q == "BSND":
+        bounds = [(b * p.S1, (b + 1) * p.S1) for b in range(p.B)]
+    else:
+        c = [0] + inp["act_q"].tolist()
+        bounds = [(c[b], c[b + 1]) for b in range(p.B)]
+    distinct = 0
+    for lo, hi in bounds:
+        sel = idx[lo:hi][valid[lo:hi]]
+        distinct += int(np.unique(sel).size)
+    io = p.rows * p.N1 * (p.D + p.Dv) * 2 + idx.size * 4 + p.rows * p.N1 * 4
+    return pairs, flops, gathered, io + distinct * (p.D + p.Dv) * 2
 
 
 def sfa_reference(args, rank):
@@ -379,7 +736,8 @@ def sfa_reference(args, rank):
 
 
 def sfa_main(args, ws, rank, local):
-    """One step = one li_sparse_attention call over the whole workload."""
+    """One step = one li_sparse_attention call over the whole workload; under
+    torchrun every rank runs its own problem of the same shape (weak scaling)."""
     import torch
 
     import sparse_attention_top_n1_b200 as li
@@ -389,18 +747,13 @@ def sfa_main(args, ws, rank, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     p, inp = sfa_workload(args.workload, rank)
-    pairs, flops, gathered, io = sfa_counts(p, inp)
+    pairs, flops, gathered, compulsory = sfa_counts(p, inp)
     d = {k: v.to(dev) for k, v in inp.items()}
     pr = li.make_sfa_params(p)
     out = torch.empty((p.rows, p.N1, p.Dv), dtype=d["query"].dtype, device=dev)
     lse = torch.empty((p.rows, p.N1), dtype=torch.float32, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    clean = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-
-    def flush_l2():
-        flush.zero_()
-        clean.sum()
+    flush_l2 = make_flush(dev)
 
     def call():
         li.li_sparse_attention(pr, d["query"], d["key"], d["value"], d["sparse_indices"], d.get("act_q"),
@@ -440,10 +793,11 @@ def sfa_main(args, ws, rank, local):
         raise SystemExit("device status 0x%x" % int(status.item()))
     peaks, peak_src = load_peaks()
     ms = total_ms / K
-    tflops = flops / (ms * 1e-3) / 1e12
-    roof = {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-            "frac": tflops / peaks["bf16_tflops"], "traffic": traffic_record(args.workload, "sfa"), "kernel": "sfa",
-            "peak_source": "bf16 burst peak (tcgen05 cuBLAS), %s; this kernel issues m16n8k16 mma.sync" % peak_src}
+    kern = roofline(ms, flops, compulsory, peaks["bf16_tflops"],
+                    "bf16 dense burst peak, %s" % peak_src, peaks["hbm_gbs"], peak_src,
+                    traffic_record(args.workload, "sfa"))
+    roof = {k: kern[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic", "peak_source")}
+    roof["kernel"] = "sfa_kernel"
     e2e = None
     if not (args.no_e2e or args.plain):
         host = {k: v.pin_memory() for k, v in inp.items()}
@@ -489,13 +843,21 @@ def sfa_main(args, ws, rank, local):
         "config": {"workload": WORKLOAD_DESC[args.workload], "rows": p.rows, "selected_pairs": pairs,
                    "l2": "flushed before every timed step (256 MiB write, then a 256 MiB read of a second buffer)",
                    "parallelism": "independent replica per GPU" if ws > 1 else "1 GPU"},
-        "effective_tflops": tflops,
+        "effective_tflops": flops / (ms * 1e-3) / 1e12,
         "gathered_gbs": gathered / (ms * 1e-3) / 1e9,
         "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+def summary(rec):
+    """The per-config entry of the JSON line."""
+    keep = ("config", "dtype", "rows", "visible_pairs", "steps", "ms_per_step", "value", "unit",
+            "effective_tflops", "stage_ms", "roofline", "kernels", "whole_call_roofline",
+            "cpu_baseline", "e2e", "gpu_launches", "clocks")
+    return {k: rec[k] for k in keep}
 
 
 def main():
@@ -507,11 +869,13 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time only --workload (no per_config records of the other configurations)")
     ap.add_argument("--no-stage-events", action="store_true",
                     help="do not record per-kernel CUDA events inside the timed steps")
     ap.add_argument("--plain", action="store_true",
-                    help="exactly W warm-up and K timed calls, no clock sampling, e2e or "
-                         "CPU baseline (a fixed launch sequence for ncu)")
+                    help="exactly W warm-up and K timed calls of --workload, no clock sampling, "
+                         "e2e, CPU baseline or per-config records (a fixed launch sequence for ncu)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -537,185 +901,45 @@ def main():
         libbuild.build()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-
-    p, inp = make_workload(args.workload, rank)
-    counts = work_counts(p, inp)
-    d = {k: v.to(dev) for k, v in inp.items()}
-    pr = li.make_params(p)
-    wsb = li.alloc_workspace(pr, dev)
-    shape = li.li_output_shape(pr)
-    idx = torch.empty(shape, dtype=torch.int32, device=dev)
-    val = torch.empty(shape, dtype=torch.float32, device=dev) if p.return_value else None
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    clean = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)   # fp32: summed without a cast
-
-    def flush_l2():
-        """Evict L2: write a buffer larger than L2, then read a second one, so
-        that the written lines are back in HBM before the next step starts and
-        the timed step does not inherit their write-back."""
-        flush.zero_()
-        clean.sum()
-    quant = bool(p.quant)
-
-    def call(q, k, w, qs, ks, aq, ak, bt, oi, ov):
-        if quant:
-            li.li_quant_indexer(pr, q, k, w, qs, ks, aq, ak, bt, oi, ov, wsb)
-        else:
-            li.li_indexer(pr, q, k, w, aq, ak, bt, oi, ov, wsb)
-
-    args_dev = (d["query"], d["key"], d["weights"], d.get("q_scale"), d.get("k_scale"),
-                d.get("act_q"), d.get("act_k"), d.get("block_table"), idx, val)
-    clocks = ClockSampler(local)
-    if not args.plain:
-        clocks.start()
-    # W warm-up steps, then more of the same until the clock sampler has seen
-    # the GPU under this load for a while (its period is 200 ms)
-    t_warm = time.perf_counter()
-    nwarm = 0
-    while nwarm < args.warmup or (not args.plain and time.perf_counter() - t_warm < 0.8):
-        flush_l2()
-        call(*args_dev)
-        nwarm += 1
-        if nwarm % 16 == 0:
-            torch.cuda.synchronize()
-    torch.cuda.synchronize()
-    flags = li.li_read_device_status(wsb)
-    if flags:
-        raise SystemExit("device status 0x%x during warm-up" % flags)
-
-    K = args.steps
-    mk = lambda: torch.cuda.Event(enable_timing=True)
-
-    def timed_steps(stage_events):
-        """K steps, L2 flushed before each outside the timed interval.  With
-        stage_events, the library records per-kernel events inside each step
-        (which keeps the kernels from overlapping their launch with the
-        previous kernel's tail, so the step itself gets a little slower)."""
-        starts = [mk() for _ in range(K)]
-        ends = [mk() for _ in range(K)]
-        prof = [[mk() for _ in range(4)] for _ in range(K)]
-        for e in [x for row in prof for x in row]:      # torch creates events lazily
-            e.record()
-        torch.cuda.synchronize()
-        barrier()
-        torch.cuda.synchronize()
-        nlaunch = 0
-        torch.cuda.nvtx.range_push("timed steps%s" % (" (stage events)" if stage_events else ""))
-        for s in range(K):
-            flush_l2()
-            if stage_events:
-                li.li_set_profile_events(prof[s])
-            torch.cuda.nvtx.range_push("step %d" % s)
-            starts[s].record()
-            call(*args_dev)
-            ends[s].record()
-            torch.cuda.nvtx.range_pop()
-            nlaunch += li.li_last_launch_count()
-        torch.cuda.nvtx.range_pop()
-        li.li_set_profile_events(None)
-        torch.cuda.synchronize()
-        barrier()
-        step_ms = [starts[s].elapsed_time(ends[s]) for s in range(K)]
-        stage = {"scheduler": [], "score": [], "topk": []}
-        if stage_events:
-            for s in range(K):
-                e = prof[s]
-                stage["scheduler"].append(e[0].elapsed_time(e[1]))
-                stage["score"].append(e[1].elapsed_time(e[2]))
-                stage["topk"].append(e[2].elapsed_time(e[3]))
-        return sum(step_ms), stage, nlaunch
-
-    # timed region 1: the job value, nothing between the kernels
-    own_ms, _, launches = timed_steps(False)
-    total_ms = allreduce_max(own_ms)
-    # timed region 2: the same steps with per-kernel events, for the roofline
-    staged_ms = 0.0
-    stage = {"scheduler": [], "score": [], "topk": []}
-    if not args.no_stage_events:
-        own_staged, stage, _ = timed_steps(True)
-        staged_ms = allreduce_max(own_staged)
-    clk = clocks.stop()
-    avg = {k: (sum(v) / len(v) if v else float("nan")) for k, v in stage.items()}
-
     peaks, peak_src = load_peaks()
-    score_tflops = counts["flops"] / (avg["score"] * 1e-3) / 1e12
-    topk_gbs = counts["topk_bytes"] / (avg["topk"] * 1e-3) / 1e9
-    tensor_peak = peaks["bf16_tflops"] * (2.0 if counts["es"] == 1 else 1.0)
-    tensor_note = ("bf16 burst peak x2 (nominal 8-bit/bf16 ratio, fp8 and int8 alike), %s" % peak_src
-                   if counts["es"] == 1 else "bf16 burst peak (fp16 has the same rate), %s" % peak_src)
-    kern = {
-        "score": {"bound": "tensor", "achieved": score_tflops, "peak": tensor_peak,
-                  "unit": "TFLOP/s", "frac": score_tflops / tensor_peak, "ms": avg["score"],
-                  "peak_source": tensor_note,
-                  "traffic": traffic_record(args.workload, "score")},
-        "topk": {"bound": "hbm", "achieved": topk_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                 "frac": topk_gbs / peaks["hbm_gbs"], "ms": avg["topk"],
-                 "peak_source": "hbm copy peak, %s" % peak_src,
-                 "traffic": traffic_record(args.workload, "topk")},
-    }
-    dom = max(("score", "topk"), key=lambda k: kern[k]["ms"])
-    roof = {k: kern[dom][k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
-    roof["kernel"] = dom
+    p8 = None if args.plain else measure_8bit_peaks(dev)
+    ctx = {"li": li, "dev": dev, "ws": ws, "rank": rank, "local": local, "peaks": peaks,
+           "peak_src": peak_src, "p8": p8, "flush": make_flush(dev)}
 
-    n = ws
-    value = job_value(p.rows, K, n, total_ms)
-    eff_tflops = n * counts["flops"] * K / (total_ms * 1e-3) / 1e12
-    whole_frac = max(counts["flops"] / (tensor_peak * 1e12),
-                     counts["compulsory_bytes"] / (peaks["hbm_gbs"] * 1e9)) / (total_ms * 1e-3 / K)
+    head = time_indexer(args.workload, args, ctx, args.steps, args.warmup, cpu_budget=12.0)
+    per_config = None
+    if ws == 1 and not (args.plain or args.no_per_config):
+        per_config = {}
+        pc_steps = max(3, min(args.steps, 10))
+        for name in CONFIGS:
+            if name == args.workload:
+                per_config[name] = summary(head)
+                continue
+            per_config[name] = summary(time_indexer(name, args, ctx, pc_steps, 3, cpu_budget=4.0))
 
-    # end to end through the C ABI with host buffers: H2D of the inputs from
-    # pinned memory, the call, D2H of the outputs, all inside the timed region
-    e2e = None
-    if not (args.no_e2e or args.plain):
-        host = {k: v.pin_memory() for k, v in inp.items()}
-        hidx = torch.empty(shape, dtype=torch.int32).pin_memory()
-        hval = torch.empty(shape, dtype=torch.float32).pin_memory() if p.return_value else None
-        h2d = sum(v.numel() * v.element_size() for v in host.values())
-        d2h = hidx.numel() * 4 + (hval.numel() * 4 if hval is not None else 0)
-        e_st = [mk() for _ in range(K + args.warmup)]
-        e_en = [mk() for _ in range(K + args.warmup)]
-        for s in range(K + args.warmup):
-            flush_l2()
-            e_st[s].record()
-            for k2, v in host.items():
-                d[k2].copy_(v, non_blocking=True)
-            call(*args_dev)
-            hidx.copy_(idx, non_blocking=True)
-            if hval is not None:
-                hval.copy_(val, non_blocking=True)
-            e_en[s].record()
-        torch.cuda.synchronize()
-        e_ms = allreduce_max(sum(e_st[s].elapsed_time(e_en[s]) for s in range(args.warmup, K + args.warmup)))
-        e2e = {"value": n * p.rows * K / (e_ms * 1e-3), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-    flags = li.li_read_device_status(wsb)
-    if flags:
-        raise SystemExit("device status 0x%x after timing" % flags)
-
-    cpu = None
-    if rank == 0 and n == 1 and not (args.no_cpu_baseline or args.plain):
-        cpu, _, _ = cpu_oracle_sample(p, inp)
-
-    dtype = {"bf16": "bf16", "fp16": "fp16", "e4m3": "fp8_e4m3", "int8": "int8"}[p.dtype_qk]
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": n, "steps": K,
-        "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
-        "config": {"workload": WORKLOAD_DESC[args.workload], "rows": p.rows,
-                   "visible_pairs": counts["pairs"], "sparse_count": p.sparse_count,
-                   "return_value": p.return_value,
+        "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": head["dtype"],
+        "data": "synthetic",
+        "config": {"workload": head["config"], "rows": head["rows"],
+                   "visible_pairs": head["visible_pairs"], "sparse_count": head["sparse_count"],
+                   "return_value": head["return_value"],
                    "l2": "flushed before every timed step (256 MiB write, then a 256 MiB read of a second buffer)",
-                   "parallelism": "independent replica per GPU" if n > 1 else "1 GPU"},
-        "ms_per_step_with_stage_events": (staged_ms / K) if staged_ms else None,
-        "effective_tflops": eff_tflops,
-        "whole_call_roofline_frac": whole_frac,
-        "roofline": roof,
-        "kernels": kern,
-        "stage_ms": avg,
-        "cpu_baseline": cpu,
-        "e2e": e2e,
-        "gpu_launches": launches,
-        "clocks": clk,
+                   "parallelism": ("query rows split over %d GPUs, balanced by visible pairs, keys replicated, "
+                                   "no data-path collective" % ws) if ws > 1 else "1 GPU"},
+        "ms_per_step_with_stage_events": head["ms_per_step_with_stage_events"],
+        "effective_tflops": head["effective_tflops"],
+        "whole_call_roofline": head["whole_call_roofline"],
+        "roofline": head["roofline"],
+        "kernels": head["kernels"],
+        "stage_ms": head["stage_ms"],
+        "cpu_baseline": head["cpu_baseline"],
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
+        "clocks": head["clocks"],
+        "tensor_peaks_8bit": p8,
+        "per_config": per_config,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -203,6 +203,9 @@ LI_API li_status li_topk(const float *scores, int64_t ld, const int32_t *row_len
  *     li_indexer with a workspace for them.
  *   - The first call on a device looks up that device's copy of the array
  *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *     The address belongs to the device's current context: a call made after
+ *     that context was destroyed and re-created (cudaDeviceReset) looks it up
+ *     again, so that call too should come before any capture.
  *   - All calls on a device share the one array and it keeps the contents of
  *     the last call.  Nothing in it has to start at zero (each call's
  *     scheduler overwrites the status and tables, and every score is written

@@ -30,6 +30,8 @@ LAYOUT = {"BSND": 0, "TND": 1, "PA_BSND": 2}
 DEV_BAD_QLEN, DEV_BAD_KLEN, DEV_BAD_BLOCK, DEV_NEG_SCALE, DEV_TIMEOUT = 1, 2, 4, 8, 16
 DEV_BAD_INDEX = 32
 INT64_MAX = (1 << 63) - 1
+# LI_NOALLOC_SCRATCH_BYTES of include/li.h: the scratch li_indexer_noalloc holds
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 EXPORTS = ("li_output_shape", "li_workspace_size", "li_indexer", "li_quant_indexer", "li_topk",
            "li_last_error", "li_read_device_status", "li_selftest_bounded_wait",

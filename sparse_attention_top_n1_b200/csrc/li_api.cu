@@ -11,8 +11,10 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "li_internal.cuh"
 #include "ptx.cuh"
@@ -425,6 +427,54 @@ li_status run(const li_params *pp, bool quant, const void *query, const void *ke
 }  // namespace
 
 namespace li {
+
+uint64_t current_context_id()
+{
+    typedef CUresult (*GetCurrentFn)(CUcontext *);
+    typedef CUresult (*GetIdFn)(CUcontext, unsigned long long *);
+    static GetCurrentFn get_current = nullptr;
+    static GetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetIdFn>(p);
+    });
+    if (!get_current || !get_id) return 0;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+    unsigned long long id = 0;
+    if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+cudaError_t set_max_dynamic_smem(const void *kern, int bytes)
+{
+    static std::mutex mu;
+    static std::map<std::pair<const void *, uint64_t>, int> done;
+    const uint64_t ctx = current_context_id();
+    if (ctx) {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = done.find({kern, ctx});
+        if (it != done.end() && it->second >= bytes) return cudaSuccess;
+    }
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    const uint64_t ctx_after = current_context_id();   // the call may have made the context current
+    if (ctx_after) {
+        std::lock_guard<std::mutex> lock(mu);
+        int &v = done[{kern, ctx_after}];
+        if (v < bytes) v = bytes;
+    }
+    return cudaSuccess;
+}
+
 // Record `msg` as the thread's last error and return `s` (for the other
 // translation units of the library).
 li_status report_error(li_status s, const char *msg) { return fail(s, "%s", msg); }

@@ -152,4 +152,13 @@ cudaError_t launch_score(const ScoreArgs &a, const Tiling &t, const CUtensorMap 
 cudaError_t launch_topk(const TopkArgs &a, cudaStream_t s);
 cudaError_t launch_wait_selftest(int32_t *status, int64_t timeout_ns, cudaStream_t s);
 
+// Unique id of the calling thread's current CUDA context (the driver's
+// cuCtxGetId), or 0 when there is none or it cannot be read.  Ids are never
+// reused within a process, so a context re-created after cudaDeviceReset
+// gets a new one.
+uint64_t current_context_id();
+// Raise `kern`'s dynamic shared-memory limit to `bytes` once per kernel and
+// context (cudaFuncSetAttribute on the first launch in a context only).
+cudaError_t set_max_dynamic_smem(const void *kern, int bytes);
+
 }  // namespace li

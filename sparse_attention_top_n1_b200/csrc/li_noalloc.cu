@@ -6,7 +6,7 @@
 // scratch array compiled into the library.  Every GPU that loads the library
 // holds LI_NOALLOC_SCRATCH_BYTES of device memory for it until the process
 // exits.  This file allocates nothing: it finds the array's device address
-// once per device and hands it to li_indexer as the workspace.
+// (once per device and context) and hands it to li_indexer as the workspace.
 #include <cstdio>
 #include <mutex>
 
@@ -24,10 +24,17 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[LI_NOALLOC_SCRA
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mu;
-void *g_scratch_addr[kMaxDevices] = {};
+struct ScratchAddr {
+    void *ptr;
+    uint64_t ctx;    // id of the context the address belongs to (0: none cached)
+};
+ScratchAddr g_scratch[kMaxDevices] = {};
 
-// The current device's address of the scratch array, looked up on the first
-// call for that device (which should precede any stream capture).
+// The current device's address of the scratch array.  It is looked up with
+// cudaGetSymbolAddress on the first call in each context of the device (the
+// first call, which should precede any stream capture, and again after a
+// cudaDeviceReset re-created the context, since the old address died with
+// the old context); later calls in the same context reuse it.
 li_status scratch_for_current_device(void **out)
 {
     int dev = -1;
@@ -35,8 +42,9 @@ li_status scratch_for_current_device(void **out)
     if (e != cudaSuccess) return li::report_error(LI_ERR_CUDA, "li_indexer_noalloc: no CUDA device");
     if (dev < 0 || dev >= kMaxDevices)
         return li::report_error(LI_ERR_CUDA, "li_indexer_noalloc: device ordinal out of range");
+    const uint64_t ctx = li::current_context_id();
     std::lock_guard<std::mutex> lock(g_setup_mu);
-    if (!g_scratch_addr[dev]) {
+    if (ctx == 0 || g_scratch[dev].ctx != ctx || !g_scratch[dev].ptr) {
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess || !p) {
@@ -45,9 +53,10 @@ li_status scratch_for_current_device(void **out)
                      cudaGetErrorString(e));
             return li::report_error(LI_ERR_CUDA, msg);
         }
-        g_scratch_addr[dev] = p;
+        g_scratch[dev].ptr = p;
+        g_scratch[dev].ctx = li::current_context_id();   // current now, if it was not before
     }
-    *out = g_scratch_addr[dev];
+    *out = g_scratch[dev].ptr;
     return LI_OK;
 }
 

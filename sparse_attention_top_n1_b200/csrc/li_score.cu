@@ -637,7 +637,7 @@ cudaError_t launch_one(const ScoreArgs &a, const CUtensorMap &qmap, const CUtens
 {
     auto kern = score_kernel<CHUNKS, N1P, KIND>;
     const size_t smem = Geometry<CHUNKS>::SMEM;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(kern), (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);

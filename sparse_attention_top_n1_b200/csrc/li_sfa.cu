@@ -33,6 +33,7 @@
 namespace li {
 li_status report_error(li_status s, const char *msg);
 void set_launch_count(int32_t n);
+cudaError_t set_max_dynamic_smem(const void *kern, int bytes);
 }  // namespace li
 
 namespace {
@@ -436,7 +437,7 @@ template <int NW, bool F16, int C>
 cudaError_t launch(const SfaArgs &a, int rows, cudaStream_t s)
 {
     auto kern = sfa_kernel<NW, F16, C>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    cudaError_t e = li::set_max_dynamic_smem(reinterpret_cast<const void *>(kern), kSmem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)rows * C);
@@ -542,8 +543,9 @@ extern "C" LI_API li_status li_sparse_attention(const li_sfa_params *p, const vo
     if (rows > 0x7FFFFFFF || key_rows > 0x7FFFFFFF || (int64_t)p->max_blocks_per_seq * p->block_size > 0x7FFFFFFF)
         return report_error(LI_ERR_SHAPE, "li_sparse_attention: more than 2^31-1 query or key rows");
     if (!aligned(query, 16) || !aligned(key, 16) || !aligned(value, 16) || !aligned(out, 16) ||
-        !aligned(sparse_indices, 4) || (lse && !aligned(lse, 4)))
-        return report_error(LI_ERR_SHAPE, "li_sparse_attention: query/key/value/out must be 16-byte aligned");
+        !aligned(sparse_indices, 4) || (lse && !aligned(lse, 4)) || (status && !aligned(status, 4)))
+        return report_error(LI_ERR_SHAPE, "li_sparse_attention: query/key/value/out must be 16-byte aligned, "
+                                          "sparse_indices/lse/status 4-byte aligned");
     li::set_launch_count(0);
     if (rows == 0) return LI_OK;
     SfaArgs a{};

@@ -942,8 +942,7 @@ size_t topk_smem_bytes(int cap, int kmax)
 cudaError_t launch_single(const TopkArgs &a, cudaStream_t s)
 {
     const size_t smem = topk_smem_bytes(a.cap, a.kmax);
-    cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(topk_kernel), (int)smem);
     if (e != cudaSuccess) return e;
     if (a.rows <= 0) return cudaSuccess;
     cudaLaunchConfig_t cfg = {};
@@ -974,7 +973,7 @@ cudaError_t launch_cluster(const TopkArgs &a, cudaStream_t s)
 {
     auto kern = topk_cluster_kernel<kMaxCluster, kTopkThreads, EPT>;
     const size_t smem = topk_cluster_smem_bytes(a.kmax);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(kern), (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)a.rows * kMaxCluster);

@@ -40,14 +40,51 @@ def test_named_workload_pairs():
 
 def test_sparse_attention_counts():
     p, x = ssfa.make_sfa(63, B=2, S1=10, S2=90, q_lens=[10, 6], N1=32, K=48, holes=0.3)
-    pairs, flops, gathered, io = bench.sfa_counts(p, x)
+    pairs, flops, gathered, compulsory = bench.sfa_counts(p, x)
     idx = x["sparse_indices"].reshape(p.rows, p.sparse_count)
     assert pairs == int((idx >= 0).sum())
     assert flops == 2.0 * p.N1 * (p.D + p.Dv) * pairs
     assert gathered == pairs * (p.D + p.Dv) * 2
-    assert io == p.rows * p.N1 * (p.D + p.Dv) * 2 + idx.numel() * 4 + p.rows * p.N1 * 4
+    # distinct selected keys per batch, counted directly
+    distinct = 0
+    for b, (lo, hi) in enumerate([(0, 10), (10, 20)]):
+        keys = set()
+        for r in range(lo, hi):
+            keys |= {int(j) for j in idx[r] if j >= 0}
+        distinct += len(keys)
+    io = p.rows * p.N1 * (p.D + p.Dv) * 2 + idx.numel() * 4 + p.rows * p.N1 * 4
+    assert compulsory == io + distinct * (p.D + p.Dv) * 2
 
 
-def test_job_value_is_whole_job_rows_over_slowest_time():
-    assert bench.job_value(1024, 20, 1, 2.0) == 1024 * 20 / 2e-3
-    assert bench.job_value(1024, 20, 4, 2.0) == 4 * 1024 * 20 / 2e-3
+def test_job_value_is_the_problems_rows_over_the_slowest_time():
+    assert bench.job_value(1024, 20, 2.0) == 1024 * 20 / 2e-3
+
+
+def test_roofline_takes_the_slower_bound():
+    # paged decode shape: 64 FLOP per byte is below the ridge point, so HBM bounds it
+    r = bench.roofline(0.2, 3.65e10, 5.72e8, 1673.8, "t", 6446.3, "h")
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert abs(r["frac"] - (5.72e8 / 6446.3e9) / 0.2e-3) < 1e-12
+    assert abs(r["achieved"] - 5.72e8 / 0.2e-3 / 1e9) < 1e-9
+    # DSA prefill shape: tensor-bound
+    r = bench.roofline(0.7, 5.5e11, 2.7e8, 1673.8, "t", 6446.3, "h")
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert abs(r["frac"] - (5.5e11 / 1673.8e12) / 0.7e-3) < 1e-12
+
+
+def test_8bit_peak_falls_back_only_when_the_measurement_is_missing_or_low():
+    peaks = {"bf16_tflops": 1600.0, "hbm_gbs": 6400.0}
+    v, src = bench.tensor_peak("e4m3", peaks, "m", {"fp8_tflops": 3100.0, "how": "x"})
+    assert v == 3100.0 and "measured in this run" in src
+    v, src = bench.tensor_peak("int8", peaks, "m", {"int8_tops": 200.0, "how": "x"})
+    assert v == 3200.0 and src.startswith("assumed")
+    v, src = bench.tensor_peak("bf16", peaks, "m", None)
+    assert v == 1600.0
+
+
+def test_default_workload_is_the_largest_configuration():
+    sizes = {}
+    for name in bench.CONFIGS:
+        p, x = bench.make_workload(name)
+        sizes[name] = bench.work_counts(p, x)["flops"]
+    assert max(sizes, key=sizes.get) == bench.DEFAULT_WORKLOAD == "quant_varlen"

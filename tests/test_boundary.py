@@ -260,14 +260,16 @@ def test_sfa_rejects_before_launch(kw, err):
 def test_sfa_pointer_checks():
     L = li.lib()
     pr = _sfa_base()
-    call = lambda q=FAKE, k=FAKE, v=FAKE, i=FAKE, aq=None, ak=None, bt=None, o=FAKE, lse=None, p=pr: \
-        li.STATUS_NAMES[L.li_sparse_attention(ctypes.byref(p), q, k, v, i, aq, ak, bt, o, lse, None, None)]
+    call = lambda q=FAKE, k=FAKE, v=FAKE, i=FAKE, aq=None, ak=None, bt=None, o=FAKE, lse=None, p=pr, st=None: \
+        li.STATUS_NAMES[L.li_sparse_attention(ctypes.byref(p), q, k, v, i, aq, ak, bt, o, lse, st, None)]
     assert call(q=None) == "LI_ERR_NULL"
     assert call(v=None) == "LI_ERR_NULL"
     assert call(i=None) == "LI_ERR_NULL"
     assert call(o=None) == "LI_ERR_NULL"
     assert call(k=FAKE + 8) == "LI_ERR_SHAPE"           # 16-byte alignment
     assert call(o=FAKE + 4) == "LI_ERR_SHAPE"
+    assert call(st=FAKE + 2) == "LI_ERR_SHAPE"           # the status word takes atomics: 4-byte aligned
+    assert call(lse=FAKE + 2) == "LI_ERR_SHAPE"
     tnd = _sfa_base(layout_q="TND", layout_kv="TND", T1=8, T2=8)
     assert call(p=tnd) == "LI_ERR_NULL"                  # TND needs the prefix sums
     pa = _sfa_base(layout_kv="PA_BSND", num_blocks=4, block_size=16, max_blocks_per_seq=2)
@@ -282,3 +284,11 @@ def test_sfa_valid_call_without_device_reports_cuda_error():
     st = li.lib().li_sparse_attention(ctypes.byref(pr), FAKE, FAKE, FAKE, FAKE, None, None, None,
                                       FAKE, None, None, None)
     assert li.STATUS_NAMES[st] == "LI_ERR_CUDA"
+
+
+def test_noalloc_scratch_size_matches_the_header():
+    import re
+    hdr = open(os.path.join(ROOT, "include", "li.h")).read()
+    m = re.search(r"#define LI_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", hdr)
+    assert m, "LI_NOALLOC_SCRATCH_BYTES not found"
+    assert li.NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))

@@ -1,10 +1,12 @@
 """The N > 1 path of bench.py, on CPU with the gloo backend (world size 2).
 
-Under torchrun every rank runs an independent problem of the same shape (weak
-scaling over independent query rows: the indexer has no data-path exchange),
-the job time is the max over ranks and rank 0 reports every rank's rows over
-that time.  These tests run two real processes to check the reduction, the
-per-rank problems and the reference arm's rank handling.
+Under torchrun the indexer problem is split by query rows (each rank a
+contiguous, pair-balanced range; the split itself is checked against the
+oracle in test_shard.py), the job time is the max over ranks and rank 0
+reports the problem's rows over that time.  The sparse attention workloads
+run one independent problem per rank.  These tests run two real processes to
+check the reduction, the per-rank row ranges and the reference arm's rank
+handling.
 """
 from __future__ import annotations
 
@@ -36,13 +38,15 @@ def _worker(rank, world, port, q):
     own_ms = [3.0, 7.5][rank]
     mx = bench.allreduce_max(own_ms, device="cpu")
     bench.barrier()
-    p, inp = bench.make_workload("tiny", rank)
-    q.put((rank, mx, p.rows, float(inp["query"].float().sum())))
+    from sparse_attention_top_n1_b200 import shard
+    p, inp = bench.make_workload("dsa_prefill")
+    pieces = shard.shard(p, world, inp.get("act_q"), inp.get("act_k"))[rank]
+    q.put((rank, mx, p.rows, [(pc.r0, pc.r1) for pc in pieces]))
     dist.barrier()
     dist.destroy_process_group()
 
 
-def test_two_gloo_ranks_reduce_max_and_draw_independent_problems():
+def test_two_gloo_ranks_reduce_max_and_split_one_problem():
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
@@ -55,10 +59,14 @@ def test_two_gloo_ranks_reduce_max_and_draw_independent_problems():
         assert pr.exitcode == 0
     (r0, mx0, rows0, s0), (r1, mx1, rows1, s1) = out
     assert mx0 == mx1 == 7.5                 # the slowest rank's time
-    assert rows0 == rows1                    # same shape on every rank
-    assert s0 != s1                          # but independent data
-    # whole-job value: all ranks' rows over the slowest rank's time
-    assert abs(bench.job_value(rows0, 10, 2, 7.5) - 2 * rows0 * 10 / 7.5e-3) < 1e-6
+    assert rows0 == rows1 == 8192            # one problem, seen by both
+    # the two ranks' ranges tile the rows; the causal triangle puts more rows on rank 0
+    spans = sorted(s0 + s1)
+    assert spans[0][0] == 0 and spans[-1][1] == 8192
+    assert all(a[1] == b[0] for a, b in zip(spans, spans[1:]))
+    assert s0[-1][1] > 4096
+    # whole-job value: the problem's rows over the slowest rank's time
+    assert abs(bench.job_value(rows0, 10, 7.5) - rows0 * 10 / 7.5e-3) < 1e-6
 
 
 def test_reference_arm_other_ranks_exit_without_work(capsys):

@@ -41,7 +41,7 @@ def test_noalloc_matches_workspace_entry_point(make):
     p, inp = make()
     d = to_device(inp)
     pr = li.make_params(p)
-    assert li.li_workspace_size(pr) <= (32 << 20)
+    assert li.li_workspace_size(pr) <= li.NOALLOC_SCRATCH_BYTES
     ref_idx, ref_val = li.indexer(pr, d["query"], d["key"], d["weights"],
                                   act_seq_q=d.get("act_q"), act_seq_k=d.get("act_k"),
                                   block_table=d.get("block_table"))
@@ -62,8 +62,55 @@ def test_noalloc_matches_workspace_entry_point(make):
 def test_noalloc_refuses_problems_beyond_its_scratch():
     p, _ = synth.make_dsa_prefill(S=8192)            # needs ~256 MiB of score rows
     pr = li.make_params(p)
-    assert li.li_workspace_size(pr) > (32 << 20)
+    assert li.li_workspace_size(pr) > li.NOALLOC_SCRATCH_BYTES
     st = li.lib().li_indexer_noalloc(ctypes.byref(pr), None, None, None, None, None, None,
                                      None, None, None)
     assert li.STATUS_NAMES[st] == "LI_ERR_WORKSPACE"
     assert "bytes of scratch" in li.li_last_error()
+
+
+def _edge_problem(over: bool):
+    """A BSND problem whose workspace is the largest at or under the scratch
+    size (over=False) or the smallest above it (over=True): rows grow one at
+    a time at a fixed key length (each row adds one fp32 score row)."""
+    S2 = 4096
+
+    def size(S1):
+        p, inp = synth.make_random(17, B=1, S1=S1, S2=S2, N1=8, sparse_count=64, ragged=False,
+                                   sparse_mode=0)
+        return li.li_workspace_size(li.make_params(p)), p, inp
+
+    lo, hi = 1, 4096                       # size(lo) <= limit < size(hi)
+    assert size(hi)[0] > li.NOALLOC_SCRATCH_BYTES
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        if size(mid)[0] <= li.NOALLOC_SCRATCH_BYTES:
+            lo = mid
+        else:
+            hi = mid
+    return size(hi if over else lo)
+
+
+def test_noalloc_at_the_limit_runs_and_one_row_more_is_refused():
+    need, p, inp = _edge_problem(over=False)
+    assert need <= li.NOALLOC_SCRATCH_BYTES
+    d = to_device(inp)
+    pr = li.make_params(p)
+    ref_idx, ref_val = li.indexer(pr, d["query"], d["key"], d["weights"],
+                                  act_seq_q=d.get("act_q"), act_seq_k=d.get("act_k"))
+    idx, val = _run_noalloc(pr, d, li.li_output_shape(pr), p.return_value)
+    np.testing.assert_array_equal(idx, ref_idx.cpu().numpy())
+    np.testing.assert_array_equal(val, ref_val.cpu().numpy())
+    need, p, inp = _edge_problem(over=True)
+    assert need > li.NOALLOC_SCRATCH_BYTES
+    d = to_device(inp)
+    pr = li.make_params(p)
+    shape = li.li_output_shape(pr)
+    idx = torch.full(shape, 5, dtype=torch.int32, device="cuda")
+    val = torch.full(shape, 5.0, dtype=torch.float32, device="cuda")
+    with pytest.raises(li.LiError) as ei:
+        li.li_indexer_noalloc(pr, d["query"], d["key"], d["weights"], d.get("act_q"),
+                              d.get("act_k"), None, idx, val)
+    assert ei.value.status == 6                          # LI_ERR_WORKSPACE
+    torch.cuda.synchronize()
+    assert bool((idx == 5).all())                        # nothing was launched

@@ -17,6 +17,8 @@ The rule (tolerance |g - o| <= atol + rtol*|o|; bf16/fp16/int8: rtol 2e-3, atol
 """
 from __future__ import annotations
 
+import os
+
 import numpy as np
 import torch
 
@@ -95,6 +97,15 @@ def check_against_oracle(p, inputs, gpu_idx, gpu_val, rows=None, nthreads=0):
         gv = gv[np.asarray(rows)] if gv is not None else None
     compare_rows(p, gi, gv, orc, rows_label=rows)
     return orc
+
+
+def check_all_rows(p, inputs, gpu_idx, gpu_val, chunk=2048):
+    """check_against_oracle on every row, `chunk` rows at a time (the oracle's
+    full score rows of a chunk are held in fp64), on all host cores."""
+    nthreads = os.cpu_count() or 1
+    for r0 in range(0, p.rows, chunk):
+        check_against_oracle(p, inputs, gpu_idx, gpu_val, rows=list(range(r0, min(p.rows, r0 + chunk))),
+                             nthreads=nthreads)
 
 
 def sample_rows(p, n_random=256, seed=0, edge=64):

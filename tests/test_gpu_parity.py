@@ -19,7 +19,7 @@ import torch
 import oracle
 import sparse_attention_top_n1_b200 as li
 import synth
-from parity import check_against_oracle, sample_rows, to_device
+from parity import check_against_oracle, check_all_rows, sample_rows, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -135,11 +135,11 @@ def test_v2_compressed_example_full():
     check_against_oracle(p, inp, gi, gv)
 
 
-def test_dsa_prefill_window_workload_sampled():
+def test_dsa_prefill_window_workload_all_rows():
     p, inp = synth.make_dsa_prefill_window()
     gi, gv, flags = run_gpu(p, inp)
     assert flags == 0
-    check_against_oracle(p, inp, gi, gv, rows=sample_rows(p, n_random=48, edge=16))
+    check_all_rows(p, inp, gi, gv)
 
 
 def test_quant_int8_readme_example_full():
@@ -151,11 +151,11 @@ def test_quant_int8_readme_example_full():
     check_against_oracle(p, inp, gi, gv)
 
 
-def test_quant_int8_varlen_sampled():
+def test_quant_int8_varlen_all_rows():
     p, inp = synth.make_quant_varlen_int8(return_value=1)
     gi, gv, flags = run_gpu(p, inp)
     assert flags == 0
-    check_against_oracle(p, inp, gi, gv, rows=sample_rows(p, n_random=64, edge=16))
+    check_all_rows(p, inp, gi, gv)
 
 
 def test_tiny_workload():
@@ -172,11 +172,11 @@ def test_cfg2_workload_full():
     check_against_oracle(p, inp, gi, gv)
 
 
-def test_dsa_prefill_workload_sampled():
+def test_dsa_prefill_workload_all_rows():
     p, inp = synth.make_dsa_prefill()
     gi, gv, flags = run_gpu(p, inp)
     assert flags == 0
-    check_against_oracle(p, inp, gi, gv, rows=sample_rows(p, n_random=96, edge=24))
+    check_all_rows(p, inp, gi, gv)
 
 
 def test_paged_decode_workload_full():
@@ -186,15 +186,11 @@ def test_paged_decode_workload_full():
     check_against_oracle(p, inp, gi, gv)
 
 
-def test_quant_varlen_workload_sampled():
+def test_quant_varlen_workload_all_rows():
     p, inp = synth.make_quant_varlen(return_value=1)
     gi, gv, flags = run_gpu(p, inp)
     assert flags == 0
-    cq = [0] + inp["act_q"].tolist()
-    rows = set(sample_rows(p, n_random=64, edge=16))
-    for b in range(p.B):                      # both ends of every sequence
-        rows |= {cq[b], cq[b] + 1, cq[b + 1] - 2, cq[b + 1] - 1}
-    check_against_oracle(p, inp, gi, gv, rows=sorted(rows))
+    check_all_rows(p, inp, gi, gv)
 
 
 # ------------------------------------------------------------------ Top-k stage alone

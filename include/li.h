@@ -80,7 +80,7 @@ typedef enum { LI_BSND = 0, LI_TND = 1, LI_PA_BSND = 2 } li_layout;
  *                  PA pool geometry; block_size a multiple of 16 in [16, 1024]
  *   key_block_stride  elements between consecutive PA blocks (0 = dense
  *                  block_size*N2*D); lets axis 0 of the pool be non-contiguous
- *   sparse_count   k, 1..2048
+ *   sparse_count   k, 1..8192 (CANN guide, "约束说明")
  *   sparse_mode    0 = every key inside the actual length; 3 = right-down causal:
  *                  key t is visible to query i of batch b iff t <= i + Sk_b - Sq_b
  *   pre_tokens, next_tokens  reserved; must be INT64_MAX

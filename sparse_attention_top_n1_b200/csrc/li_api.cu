@@ -82,8 +82,6 @@ li_status check_params(const li_params *pp, bool quant)
     if (p.N1 < 1 || p.N1 > 64) return fail(LI_ERR_SHAPE, "N1 must be in [1, 64]");
     if (p.sparse_count < 1 || p.sparse_count > 8192)
         return fail(LI_ERR_SHAPE, "sparse_count must be in [1, 8192]");
-    if (p.sparse_count > 2048)
-        return fail(LI_ERR_UNSUPPORTED, "sparse_count above 2048 is not built yet");
     if (p.sparse_mode != 0 && p.sparse_mode != 3)
         return fail(LI_ERR_SHAPE, "sparse_mode must be 0 or 3");
     if (p.pre_tokens != kInt64Max || p.next_tokens != kInt64Max)
@@ -539,8 +537,7 @@ li_status li_topk(const float *scores, int64_t ld, const int32_t *row_len, int32
     g_launches = 0;
     if (!scores || !sparse_indices) return fail(LI_ERR_NULL, "scores and sparse_indices are required");
     if (rows < 0) return fail(LI_ERR_SHAPE, "rows must be >= 0");
-    if (k < 1 || k > 2048) return fail(k > 8192 || k < 1 ? LI_ERR_SHAPE : LI_ERR_UNSUPPORTED,
-                                       "k must be in [1, 2048]");
+    if (k < 1 || k > 8192) return fail(LI_ERR_SHAPE, "k must be in [1, 8192]");
     if (ld < 1 || ld % 4 || ld > kInt32Max) return fail(LI_ERR_SHAPE, "ld must be a positive multiple of 4");
     if (!aligned(scores, 16)) return fail(LI_ERR_SHAPE, "scores must be 16-byte aligned");
     TopkArgs ta{};

@@ -156,12 +156,12 @@ struct TopkShared {
 // Keys j < fa and j >= fc are forced (sink tokens and local window): they
 // take part in the selection as the largest possible key and are ordered by
 // their real key (fa = 0, fc = n: none forced).
-template <int NT>
+template <int NT, int KMAX>
 __device__ void radix_topk(const RowSrc &src, int n, int k, int m, const TopkSmem &s,
                            TopkShared &sh, int32_t *oidx, float *oval, int fa, int fc)
 {
     constexpr int kTopkThreads = NT, kWarps = NT / 32;
-    constexpr int kSortMaxRounds = 2048 / NT;       // rounds of 32 per warp for kmax <= 2048
+    constexpr int kSortMaxRounds = KMAX / NT;       // rounds of 32 per warp for kmax <= KMAX
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int n4 = (n + 3) >> 2;
     uint32_t *hist = s.hist, *keyA = s.keyA, *keyB = s.keyB;
@@ -504,6 +504,7 @@ __device__ bool bucket_topk(const RowSrc &src, int n, int k, int m, int kmax, co
     return true;
 }
 
+template <int KMAX>
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a)
 {
     extern __shared__ __align__(16) uint8_t smem[];
@@ -600,7 +601,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a)
     const int fa = a.init_num < n ? a.init_num : n;
     const int fc = (n - a.local_num) > fa ? n - a.local_num : fa;
     if (fa > 0 || fc < n || !bucket_topk(src, n, k, m, a.kmax, s, sh, oidx, oval))
-        radix_topk<kTopkThreads>(src, n, k, m, s, sh, oidx, oval, fa, fc);
+        radix_topk<kTopkThreads, KMAX>(src, n, k, m, s, sh, oidx, oval, fa, fc);
 }
 
 // Number of candidate keys of a row: the visible prefix of the batch's keys
@@ -678,9 +679,10 @@ constexpr int kCBuckets = 2048;      // 52 KB per CTA: the 512 CTAs of 64 long r
 // (order-preserving key << 32) | ~index, so that a larger word means a larger
 // value or, for equal values, a lower index.
 // Four CTAs per SM (registers capped at 32), so the 512 CTAs of 64 long rows
-// run as one wave.
-template <int C, int NT, int EPT>
-__global__ void __launch_bounds__(NT, 4) topk_cluster_kernel(TopkArgs a)
+// run as one wave; with k above 2048 the selection buffers allow one CTA per
+// SM, and the register cap is lifted.
+template <int C, int NT, int EPT, int KMAX>
+__global__ void __launch_bounds__(NT, KMAX > 2048 ? 1 : 4) topk_cluster_kernel(TopkArgs a)
 {
     constexpr int G = EPT / 4;                  // float4 groups per thread
     constexpr int PER_T = kCBuckets / NT;        // buckets per thread in the scan
@@ -729,7 +731,7 @@ __global__ void __launch_bounds__(NT, 4) topk_cluster_kernel(TopkArgs a)
         full.g = grow;
         full.c = nullptr;
         full.n = n;
-        radix_topk<NT>(full, n, k, m, s, sh, oidx, oval, fa, fc);
+        radix_topk<NT, KMAX>(full, n, k, m, s, sh, oidx, oval, fa, fc);
     };
     if (n > C * NT * EPT || fa > 0 || fc < n) {   // too long, or keys forced in
         if (rank == 0) radix_row();
@@ -939,10 +941,11 @@ size_t topk_smem_bytes(int cap, int kmax)
            (cache > pingpong ? cache : pingpong);
 }
 
+template <int KMAX>
 cudaError_t launch_single(const TopkArgs &a, cudaStream_t s)
 {
     const size_t smem = topk_smem_bytes(a.cap, a.kmax);
-    cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(topk_kernel), (int)smem);
+    cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(topk_kernel<KMAX>), (int)smem);
     if (e != cudaSuccess) return e;
     if (a.rows <= 0) return cudaSuccess;
     cudaLaunchConfig_t cfg = {};
@@ -955,7 +958,7 @@ cudaError_t launch_single(const TopkArgs &a, cudaStream_t s)
     attr[0].val.programmaticStreamSerializationAllowed = a.standalone ? 0 : 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, topk_kernel, a);
+    return cudaLaunchKernelEx(&cfg, topk_kernel<KMAX>, a);
 }
 
 // Shared memory of one cluster CTA: bucket counts and cursors, the selected
@@ -968,10 +971,10 @@ size_t topk_cluster_smem_bytes(int kmax)
            (tail_bucket > tail_radix ? tail_bucket : tail_radix) * 4;
 }
 
-template <int EPT>
+template <int EPT, int KMAX>
 cudaError_t launch_cluster(const TopkArgs &a, cudaStream_t s)
 {
-    auto kern = topk_cluster_kernel<kMaxCluster, kTopkThreads, EPT>;
+    auto kern = topk_cluster_kernel<kMaxCluster, kTopkThreads, EPT, KMAX>;
     const size_t smem = topk_cluster_smem_bytes(a.kmax);
     cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(kern), (int)smem);
     if (e != cudaSuccess) return e;
@@ -998,11 +1001,14 @@ cudaError_t launch_cluster(const TopkArgs &a, cudaStream_t s)
 cudaError_t launch_topk(const TopkArgs &a, cudaStream_t s)
 {
     if (a.rows <= 0) return cudaSuccess;
-    if (a.ld <= a.cap) return launch_single(a, s);
+    // k up to 2048 (the common case) keeps the radix sort's register rounds
+    // small; larger k (up to 8192) takes the wide instances
+    const bool big = a.kmax > 2048;
+    if (a.ld <= a.cap) return big ? launch_single<8192>(a, s) : launch_single<2048>(a, s);
     const int64_t per_thread = (a.ld + (int64_t)kMaxCluster * kTopkThreads - 1) / ((int64_t)kMaxCluster * kTopkThreads);
-    if (per_thread <= 8) return launch_cluster<8>(a, s);
-    if (per_thread <= 16) return launch_cluster<16>(a, s);
-    return launch_cluster<32>(a, s);
+    if (per_thread <= 8) return big ? launch_cluster<8, 8192>(a, s) : launch_cluster<8, 2048>(a, s);
+    if (per_thread <= 16) return big ? launch_cluster<16, 8192>(a, s) : launch_cluster<16, 2048>(a, s);
+    return big ? launch_cluster<32, 8192>(a, s) : launch_cluster<32, 2048>(a, s);
 }
 
 }  // namespace li

@@ -91,7 +91,6 @@ BAD = [
     (dict(D=96), "LI_ERR_SHAPE"),
     (dict(sparse_count=0), "LI_ERR_SHAPE"),
     (dict(sparse_count=8193), "LI_ERR_SHAPE"),
-    (dict(sparse_count=3072), "LI_ERR_UNSUPPORTED"),
     (dict(sparse_mode=1), "LI_ERR_SHAPE"),
     (dict(pre_tokens=5), "LI_ERR_SHAPE"),
     (dict(next_tokens=0), "LI_ERR_SHAPE"),
@@ -182,7 +181,7 @@ def test_topk_checks():
     L = li.lib()
     assert li.STATUS_NAMES[L.li_topk(FAKE, 6, None, 2, 4, FAKE, None, None)] == "LI_ERR_SHAPE"
     assert li.STATUS_NAMES[L.li_topk(FAKE, 8, None, 2, 0, FAKE, None, None)] == "LI_ERR_SHAPE"
-    assert li.STATUS_NAMES[L.li_topk(FAKE, 8, None, 2, 4096, FAKE, None, None)] == "LI_ERR_UNSUPPORTED"
+    assert li.STATUS_NAMES[L.li_topk(FAKE, 8, None, 2, 8193, FAKE, None, None)] == "LI_ERR_SHAPE"
     assert li.STATUS_NAMES[L.li_topk(None, 8, None, 2, 4, FAKE, None, None)] == "LI_ERR_NULL"
 
 

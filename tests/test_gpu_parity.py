@@ -214,7 +214,11 @@ def _topk_reference(rows_np, lens, k):
                                        (4096, 1024, "levels"), (16384, 2048, "levels"),
                                        (2048, 2048, "levels"), (5000, 700, "constant"),
                                        (65536, 2048, "levels"), (70000, 1, "normal"),
-                                       (140000, 2048, "normal"), (20000, 2048, "constant")])
+                                       (140000, 2048, "normal"), (20000, 2048, "constant"),
+                                       (16384, 8192, "normal"), (12000, 4096, "levels"),
+                                       (9000, 8192, "quarters"), (65536, 8192, "normal"),
+                                       (40000, 4096, "levels"), (140000, 8192, "normal"),
+                                       (30000, 8192, "constant")])
 def test_topk_stage_exact(ld, k, kind):
     """Exact against a lexsort reference.  'quarters' (values on a 0.25 grid,
     every 7th -0.0) and 'constant' rows force the radix fallback; 'levels'
@@ -302,3 +306,27 @@ def test_repeat_calls_are_deterministic():
     b = run_gpu(p, inp)
     np.testing.assert_array_equal(a[0], b[0])
     np.testing.assert_array_equal(a[1], b[1])
+
+
+# ------------------------------------------------------------------ sparse_count above 2048
+
+@pytest.mark.parametrize("k", [4096, 8192])
+def test_large_sparse_count_decode_rows(k):
+    """sparse_count up to 8192 (CANN guide, "约束说明"): decode-length paged
+    rows of 16 k to 65 k keys, every row against the oracle."""
+    p, inp = synth.make_paged_decode(seed=40 + k, B=6, lo=16384, hi=65536, return_value=1)
+    p.sparse_count = k
+    gi, gv, flags = run_gpu(p, inp)
+    assert flags == 0
+    check_against_oracle(p, inp, gi, gv)
+
+
+@pytest.mark.parametrize("k", [4096, 8192])
+def test_large_sparse_count_causal_prefill(k):
+    """Right-down causal prefill with k of 4096 and 8192: rows shorter than k
+    are sorted whole, longer ones selected; sampled rows of both kinds."""
+    p, inp = synth.make_dsa_prefill(seed=41 + k, S=12288, return_value=1)
+    p.sparse_count = k
+    gi, gv, flags = run_gpu(p, inp)
+    assert flags == 0
+    check_against_oracle(p, inp, gi, gv, rows=sample_rows(p, n_random=48, edge=8, seed=k))

@@ -1,4 +1,5 @@
-// li_sfa.cu -- sparse attention over the indexer's selected keys.
+// li_sfa.cu -- sparse attention over the indexer's selected keys, on the
+// 5th-generation tensor cores.
 //
 // The consumer of the indexer's output (CANN TileLang LightningIndexer guide,
 // section "LightningIndexer 在稀疏注意力中的地位": the index tensor names, for
@@ -9,15 +10,36 @@
 //     lse_h = log sum_{j in J} exp(scale * q_h . k_j)
 //
 // One CTA per query row (or, when rows are few, a cluster of up to 8 CTAs per
-// row, each taking a share of its keys), one warp per 16 heads.  The row's
-// selected keys are taken 64 at a time: their K and V rows are gathered from
-// wherever the index points (BSND, TND or a paged pool) into shared memory
-// with 16-byte cp.async copies, double-buffered against the math; S = Q K^T
-// and O += P V run on the tensor cores (m16n8k16, fp32 accumulation) with the
-// softmax kept online in registers (running max and sum per head, the
-// FlashAttention recurrence), so the selected keys are read once and nothing
-// but the output is written.  The weights enter P V rounded to the input
-// type and the normaliser sums the same rounded values.
+// row, each taking a share of its keys, merged through distributed shared
+// memory), two CTAs per SM, warp-specialised; the row's selected keys are
+// taken 64 at a time:
+//   warps 0-1  resolve each slot to a key row (batch offset, or the block
+//              table for a paged pool; an empty or invalid slot becomes a
+//              masked zero row) and gather the 64 key rows and 64 value rows
+//              with 16-byte cp.async copies, one 256-byte row per half warp
+//              and instruction, into two-stage key and value rings in the
+//              128-byte-swizzled layout the tensor core reads; each thread's
+//              arrival on a stage's full barrier is deferred by the copy unit
+//              until its copies have landed; the tile's slot-validity mask
+//              travels with its key stage;
+//   warp 2     issues S = Q K^T on tcgen05.mma (M = the heads, 64 or 128
+//              rows with zero rows for N1 < 64; N = 64 keys; K = D = 128)
+//              into one of two tensor-memory buffers, one tile ahead of
+//              O += P V (A = the weights, K-major; B = the value tile read
+//              MN-major from its gathered layout; fp32 accumulation in
+//              tensor memory);
+//   warps 3-6  the softmax: each reads its quarter of S out of tensor memory
+//              (M = 64: four threads per head with the 16-lane load shape,
+//              combined by two shuffles; M = 128: one thread per head), scales
+//              the logits into the log2 domain, masks empty slots, rounds the
+//              weights exp2(s - m) to the input type and writes them to a
+//              double-buffered shared-memory tile (the normaliser sums the
+//              same rounded values, so the output stays a convex combination
+//              of values); the running max m moves only when a tile's max
+//              beats it by more than 2^8, and only then is O rescaled in
+//              tensor memory, so the weights stay below 256 and O is touched
+//              rarely.
+// out = O / l and lse = ln 2 * (m + log2 l) are written once per row.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -29,6 +51,7 @@
 #include <cstdint>
 
 #include "li.h"
+#include "ptx.cuh"
 
 namespace li {
 li_status report_error(li_status s, const char *msg);
@@ -38,16 +61,17 @@ cudaError_t set_max_dynamic_smem(const void *kern, int bytes);
 
 namespace {
 
-constexpr int kTile = 64;                 // selected keys per tile
+using namespace li;
+
 constexpr int kHd = 128;                  // D = Dv
-constexpr int kRowBytes = kHd * 2;        // one key or value row
-constexpr int kChunks = kRowBytes / 16;   // 16-byte chunks per row
-constexpr int kTileBytes = kTile * kRowBytes;
-constexpr int kRowMapBytes = 2 * kTile * 4;    // [2][kTile] key row of each slot
-constexpr int kMergeBytes = 2 * 128 * 4;       // a cluster's per-head (max, sum) partials
-constexpr int kMaskBytes = 16;                 // [2][2] slot-validity bits
-constexpr int kSmem = 4 * kTileBytes + kRowMapBytes + kMergeBytes + kMaskBytes + 128;
-constexpr int kMaxSplit = 8;             // CTAs (one cluster) sharing a row's keys
+constexpr int kSlots = 64;                // selected keys per tile: the N of S, the K of P.V
+constexpr int kThreads = 224;             // two producer warps, MMA issuer, four softmax warps
+constexpr int kProducers = 64;            // one producer thread per slot of a tile
+constexpr int kKStages = 2, kVStages = 2;
+constexpr int kStageBytes = kSlots * kHd * 2;   // one key or value tile: two 64-column planes
+constexpr int kPlane = kSlots * 128;            // one 64-column plane of a tile
+constexpr int kMaxSplit = 8;              // CTAs (one cluster) sharing a row's keys
+constexpr float kRescaleLog2 = 8.f;       // the running max moves when a tile beats it by 2^8
 
 struct SfaArgs {
     const uint16_t *q, *k, *v;
@@ -62,50 +86,49 @@ struct SfaArgs {
     float scale_log2;                     // softmax scale * log2(e)
 };
 
-__device__ __forceinline__ uint32_t smem_addr(const void *p)
+// Shared memory of one CTA (byte offsets from a 1024-byte aligned base).  Q,
+// the key and value tiles and the weights are stored as 128-byte rows in
+// 64-column planes, 16-byte chunk c of row r at chunk position c ^ (r & 7)
+// (the 128-byte swizzle of TMA and of the tensor core's descriptors).
+template <int M>
+struct Layout {
+    static constexpr int QPLANE = M * 128;                  // M rows x 64 columns of 16 bits
+    static constexpr int Q = 0;                             // [2][M][128 B]
+    static constexpr int K = Q + 2 * QPLANE;                // [kKStages][2][64][128 B]
+    static constexpr int V = K + kKStages * kStageBytes;    // [kVStages][2][64][128 B]
+    static constexpr int P = V + kVStages * kStageBytes;    // [2][M][128 B]: weights, 64 keys along K
+    static constexpr int MASK = P + 2 * QPLANE;             // uint32 [kKStages][2]
+    static constexpr int BARS = MASK + 32;                  // mbarriers
+    static constexpr int NBARS = 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 2;
+    static constexpr int TSLOT = BARS + NBARS * 8;
+    static constexpr int MERGE = TSLOT + 16;                // float [2][128]: a cluster's (m, l)
+    static constexpr int END = MERGE + 2 * 128 * 4;
+    static constexpr int BYTES = END + 1024;                // + alignment of the base
+};
+
+__device__ __forceinline__ int32_t clampi(int64_t v, int64_t lo, int64_t hi)
 {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+    return (int32_t)(v < lo ? lo : (v > hi ? hi : v));
 }
 
-// 16-byte global->shared copy; src_bytes = 0 fills the destination with zeros
+// Offset of 16-byte chunk `ch` (0..15) of row `r` in a two-plane tile.
+__device__ __forceinline__ uint32_t chunk_off(int r, int ch, int plane_bytes)
+{
+    return (uint32_t)((ch >> 3) * plane_bytes + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
+}
+
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
 {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
                  : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
+// Arrive on `bar` once all earlier cp.async copies of this thread have landed;
+// the arrival counts towards the barrier's expected count (no increment).
+__device__ __forceinline__ void cp_async_arrive(uint64_t *bar)
 {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
-}
-
-template <bool F16>
-__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
-{
-    if constexpr (F16)
-        asm volatile(
-            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-            "{%0,%1,%2,%3};"
-            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-    else
-        asm volatile(
-            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-            "{%0,%1,%2,%3};"
-            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 template <bool F16>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi)
@@ -133,36 +156,96 @@ __device__ __forceinline__ float unpack_hi(uint32_t v)
     else return __uint_as_float(v & 0xFFFF0000u);
 }
 
-// Byte offset of 16-byte chunk `ch` of row `r` in a tile: rows of 256 B, the
-// low three bits of the chunk index XOR-ed with the row so that the eight
-// rows an ldmatrix phase reads sit in eight different bank groups.
-__device__ __forceinline__ uint32_t tile_off(int r, int ch)
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Columns 16*CH .. 16*CH+15 of this warp's lanes into r[16*CH ..].
+template <int CH, int N>
+__device__ __forceinline__ void tmem_ld16_into(uint32_t taddr, uint32_t (&r)[N])
 {
-    return (uint32_t)(r * kRowBytes + ((ch ^ (r & 7)) << 4));
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[16 * CH + 0]), "=r"(r[16 * CH + 1]), "=r"(r[16 * CH + 2]), "=r"(r[16 * CH + 3]),
+          "=r"(r[16 * CH + 4]), "=r"(r[16 * CH + 5]), "=r"(r[16 * CH + 6]), "=r"(r[16 * CH + 7]),
+          "=r"(r[16 * CH + 8]), "=r"(r[16 * CH + 9]), "=r"(r[16 * CH + 10]), "=r"(r[16 * CH + 11]),
+          "=r"(r[16 * CH + 12]), "=r"(r[16 * CH + 13]), "=r"(r[16 * CH + 14]), "=r"(r[16 * CH + 15])
+        : "r"(taddr + 16 * CH));
 }
 
-__device__ __forceinline__ int32_t clampi(int64_t v, int64_t lo, int64_t hi)
+// 16 lanes x 256 bits, 8 repetitions (64 columns): thread t gets lanes
+// t/4 and t/4 + 8, columns 8j + 2(t%4) and 8j + 2(t%4) + 1 in r[4j .. 4j+3]
+// (lane t/4: r[4j], r[4j+1]; lane t/4 + 8: r[4j+2], r[4j+3]).
+__device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t (&r)[32])
 {
-    return (int32_t)(v < lo ? lo : (v > hi ? hi : v));
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
 }
 
-// C > 1: a cluster of C CTAs shares one row; CTA `part` takes its share of the
-// row's key tiles, and the C partial (max, sum, O) triples are merged through
+__device__ __forceinline__ void tmem_st_16x256b_x8(uint32_t taddr, const uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x256b.x8.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+        "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+        "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+// 2^x on the special-function unit (relative error about 2^-22, far below
+// the 16-bit rounding the weights get next); 2^-inf = 0.
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Bounded wait on an mbarrier phase; an expired wait flags LI_DEV_TIMEOUT and
+// the caller goes on (results are then undefined; the context stays usable).
+__device__ __forceinline__ void wait_phase(uint64_t *bar, uint32_t parity, int32_t *status)
+{
+    // the waiting thread is suspended in hardware (up to 1 us per try) until
+    // the phase completes, instead of spinning on the issue slots
+    if (mbar_try_wait(bar, parity)) return;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait_sleep(bar, parity, 1000u)) {
+        if ((int64_t)(global_timer_ns() - t0) > 2000000000LL) {
+            if (status) atomicOr(status, LI_DEV_TIMEOUT);
+            return;
+        }
+    }
+}
+
+// M = tensor-core rows (heads, zero-padded to 64 when N1 < 64); C > 1: a
+// cluster of C CTAs shares one row, CTA `part` taking its share of the row's
+// key tiles; the C partial (max, sum, O) triples are merged through
 // distributed shared memory, so no global scratch is needed.
-template <int NW, bool F16, int C>
-__global__ void __launch_bounds__(32 * NW) sfa_kernel(const SfaArgs a)
+template <int M, bool F16, int C>
+__global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const SfaArgs a)
 {
-    static_assert(kChunks == 16, "row chunk arithmetic assumes 256-byte rows");
-    constexpr int NT = 32 * NW;
+    using L = Layout<M>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-    uint8_t *sK = base;                                      // [2] key tiles
-    uint8_t *sV = base + 2 * kTileBytes;                     // [2] value tiles
-    int32_t *sRow = reinterpret_cast<int32_t *>(base + 4 * kTileBytes);   // [2][kTile] key row, -1 = none
-    uint32_t *sMask = reinterpret_cast<uint32_t *>(base + 4 * kTileBytes + kRowMapBytes + kMergeBytes);
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint32_t *sMask = reinterpret_cast<uint32_t *>(base + L::MASK);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base + L::BARS);
+    uint64_t *kfull = bars, *kempty = bars + kKStages;
+    uint64_t *vfull = bars + 2 * kKStages, *vempty = vfull + kVStages;
+    uint64_t *sfull = vempty + kVStages, *sfree = sfull + 2;
+    uint64_t *pfull = sfree + 2, *pvdone = pfull + 2;     // per weights buffer
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(base + L::TSLOT);
+    const uint32_t sbase = smem_u32(base);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, c = lane & 3;
     const int row = blockIdx.x / C;
     const int part = C > 1 ? (int)(blockIdx.x % C) : 0;   // rank in the cluster
 
@@ -198,251 +281,521 @@ __global__ void __launch_bounds__(32 * NW) sfa_kernel(const SfaArgs a)
         Sk = clampi(a.act_k[b], 0, (int64_t)a.max_blocks_per_seq * a.block_size);
     }
     const bool valid_row = i >= 0 && i < Sq;      // uniform over the CTA
-
-    // ---- this warp's 16 heads of the query as m16n8k16 A fragments
-    uint32_t qf[8][4];
-    {
-        const uint16_t *qh = a.q + ((int64_t)row * a.N1 + warp * 16) * kHd;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            const int d = kk * 16 + 2 * c;
-            qf[kk][0] = *reinterpret_cast<const uint32_t *>(qh + g * kHd + d);
-            qf[kk][1] = *reinterpret_cast<const uint32_t *>(qh + (g + 8) * kHd + d);
-            qf[kk][2] = *reinterpret_cast<const uint32_t *>(qh + g * kHd + d + 8);
-            qf[kk][3] = *reinterpret_cast<const uint32_t *>(qh + (g + 8) * kHd + d + 8);
-        }
-    }
-
-    const int32_t *irow = a.idx + (int64_t)row * a.K;
-    // slot r of tile t: the key/value row its index names, or -1
-    auto resolve = [&](int t, int buf) -> int {
-        int ok = 0;
-        for (int r = tid; r < kTile; r += NT) {    // one CTA may have fewer threads than slots
-            const int j = t * kTile + r;
-            int kr = -1;
-            if (j < a.K) {
-                const int e = irow[j];
-                if (e >= 0 && e < Sk) {
-                    if (a.layout_kv == LI_PA_BSND) {
-                        const int id = a.block_table[(int64_t)b * a.max_blocks_per_seq + e / a.block_size];
-                        if (id >= 0 && id < a.num_blocks) kr = id * a.block_size + e % a.block_size;
-                        else if (a.status) atomicOr(a.status, LI_DEV_BAD_BLOCK);
-                    } else {
-                        kr = (int)(k_off + e);
-                    }
-                } else if (e != -1 && a.status) {
-                    atomicOr(a.status, LI_DEV_BAD_INDEX);
-                }
-            }
-            sRow[buf * kTile + r] = kr;
-            ok |= kr >= 0;
-            // whole warps run this loop (kTile is a multiple of 32)
-            const unsigned bal = __ballot_sync(0xffffffffu, kr >= 0);
-            if ((r & 31) == 0) sMask[buf * 2 + (r >> 5)] = bal;
-        }
-        return ok;
-    };
-    // gather the tile's key and value rows (zeros for empty slots)
-    auto issue = [&](int buf) {
-        const uint32_t kd = smem_addr(sK + buf * kTileBytes), vd = smem_addr(sV + buf * kTileBytes);
-        for (int ci = tid; ci < kTile * kChunks; ci += NT) {
-            const int r = ci >> 4, ch = ci & 15;
-            const int kr = sRow[buf * kTile + r];
-            const int64_t off = (int64_t)(kr < 0 ? 0 : kr) * kHd + ch * 8;
-            const uint32_t n = kr < 0 ? 0u : 16u;
-            cp_async16(kd + tile_off(r, ch), a.k + off, n);
-            cp_async16(vd + tile_off(r, ch), a.v + off, n);
-        }
-        cp_async_commit();
-    };
-
-    float o[16][4];
-#pragma unroll
-    for (int dn = 0; dn < 16; ++dn) o[dn][0] = o[dn][1] = o[dn][2] = o[dn][3] = 0.f;
-    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
-
-    const int nt_all = valid_row ? (a.K + kTile - 1) / kTile : 0;
+    const int nt_all = valid_row ? (a.K + kSlots - 1) / kSlots : 0;
     const int t_begin = nt_all * part / C, t_end = nt_all * (part + 1) / C;
-    int any_cur = 0;
-    if (t_begin < t_end) {
-        any_cur = __syncthreads_or(resolve(t_begin, 0));
-        if (any_cur) issue(0);
-        else cp_async_commit();
-    }
-    for (int t = t_begin; t < t_end; ++t) {
-        const int buf = (t - t_begin) & 1;
-        int any_next = 0;
-        if (t + 1 < t_end) {
-            any_next = __syncthreads_or(resolve(t + 1, buf ^ 1));
-            if (any_next) issue(buf ^ 1);
-            else cp_async_commit();
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
+    const int ntl = t_end - t_begin;              // this CTA's tiles
+
+    if (tid == 0) {
+        for (int s = 0; s < kKStages; ++s) {
+            mbar_init(&kfull[s], kProducers + 2); // every producer thread's copies, the two mask words
+            mbar_init(&kempty[s], 1 + 4);         // the S commit and the four softmax warps
         }
-        __syncthreads();
-        if (any_cur) {
-            const uint32_t kb = smem_addr(sK + buf * kTileBytes), vb = smem_addr(sV + buf * kTileBytes);
-            const uint64_t valid = (uint64_t)sMask[buf * 2] | ((uint64_t)sMask[buf * 2 + 1] << 32);
-            // S = Q K^T for 16 heads x 64 keys
-            float s[8][4];
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-#pragma unroll
-                for (int np = 0; np < 4; ++np) {
-                    const int key = np * 16 + (lane & 7) + ((lane >> 4) << 3);
-                    const int ch = kk * 2 + ((lane >> 3) & 1);
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4(kb + tile_off(key, ch), b0, b1, b2, b3);
-                    mma16816<F16>(s[2 * np], qf[kk], b0, b1);
-                    mma16816<F16>(s[2 * np + 1], qf[kk], b2, b3);
-                }
+        for (int s = 0; s < kVStages; ++s) {
+            mbar_init(&vfull[s], kProducers);     // every producer thread's copies
+            mbar_init(&vempty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sfull[s], 1);
+            mbar_init(&sfree[s], 4);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&pfull[s], 4);
+            mbar_init(&pvdone[s], 1);
+        }
+        fence_mbarrier_init();
+    }
+    if (warp == 2) tmem_alloc(tslot, 256);        // S: two buffers of 64 columns; O: 128-255
+    // Q into shared memory (heads beyond N1 are zero rows)
+    for (int e = tid; e < M * 16; e += kThreads) {
+        const int r = e >> 4, ch = e & 15;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (r < a.N1 && valid_row) v = *reinterpret_cast<const uint4 *>(a.q + ((int64_t)row * a.N1 + r) * kHd + ch * 8);
+        *reinterpret_cast<uint4 *>(base + L::Q + chunk_off(r, ch, L::QPLANE)) = v;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tslot;
+    const uint32_t tO = tmem + 128;
+    const int32_t *irow = a.idx + (int64_t)row * a.K;
+    const uint16_t *kv_k = a.k, *kv_v = a.v;
+
+    if (warp < 2) {
+        // ------------------------------------------------------------ producers
+        // thread p resolves slot p of every tile to its key row (index loads
+        // two tiles ahead, block-table loads one tile ahead, so no copy waits
+        // on a dependent load); the rows are then copied by half warps, 16
+        // threads x 16 bytes covering one 256-byte key or value row per
+        // copy instruction (fully used 32-byte sectors), zeros for an empty
+        // slot.  Each stage is signalled by the copies themselves: the
+        // thread's arrival on the stage's full barrier is deferred by the
+        // copy unit until all its earlier copies have landed.
+        const int sp = tid;                      // slot of this thread
+        const bool pa = a.layout_kv == LI_PA_BSND;
+        const int64_t bt_row = (int64_t)b * a.max_blocks_per_seq;
+        auto load_idx = [&](int t) -> int {      // index of this slot in tile t (or -1)
+            const int j = t * kSlots + sp;
+            return (t < t_end && j < a.K) ? irow[j] : -1;
+        };
+        auto load_blk = [&](int e) -> int {      // block id behind a valid index
+            return (pa && e >= 0 && e < Sk) ? a.block_table[bt_row + e / a.block_size] : 0;
+        };
+        auto row_of = [&](int e, int id) -> int {  // key row, or -1 (flags bad entries)
+            if (e >= 0 && e < Sk) {
+                if (!pa) return (int)(k_off + e);
+                if (id >= 0 && id < a.num_blocks) return id * a.block_size + e % a.block_size;
+                if (a.status) atomicOr(a.status, LI_DEV_BAD_BLOCK);
+                return -1;
             }
-            // online softmax in the log2 domain; rows g (e = 0, 1) and g + 8 (e = 2, 3)
+            if (e != -1 && a.status) atomicOr(a.status, LI_DEV_BAD_INDEX);
+            return -1;
+        };
+        int e_cur = load_idx(t_begin), e_nxt = load_idx(t_begin + 1);
+        int d_cur = load_blk(e_cur);
+        for (int u = 0; u < ntl; ++u) {
+            const int t = t_begin + u;
+            const int r = row_of(e_cur, d_cur);
+            const int d_nxt = load_blk(e_nxt);   // in flight while this tile's copies are issued
+            const int e_far = load_idx(t + 2);
+            const unsigned ok = __ballot_sync(0xffffffffu, r >= 0);
+            int rr[16];                          // rows of slots 32w + 2i + lane/16: one 256-byte row per half warp
+#pragma unroll
+            for (int i = 0; i < 16; ++i) rr[i] = __shfl_sync(0xffffffffu, r, 2 * i + (lane >> 4));
+            const int ks = u % kKStages, vs = u % kVStages;
+            // keys of tile u and its validity mask (read by the softmax warps after kfull)
+            wait_phase(&kempty[ks], ((u / kKStages) & 1) ^ 1u, a.status);
+            if (lane == 0) {
+                sMask[ks * 2 + warp] = ok;
+                mbar_arrive(&kfull[ks]);
+            }
+            const uint32_t kd = sbase + L::K + ks * kStageBytes;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                cp_async16(kd + chunk_off(32 * warp + 2 * i + (lane >> 4), lane & 15, kPlane),
+                           kv_k + (int64_t)(rr[i] < 0 ? 0 : rr[i]) * kHd + (lane & 15) * 8, rr[i] < 0 ? 0u : 16u);
+            cp_async_arrive(&kfull[ks]);
+            // values of tile u
+            wait_phase(&vempty[vs], ((u / kVStages) & 1) ^ 1u, a.status);
+            const uint32_t vd = sbase + L::V + vs * kStageBytes;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                cp_async16(vd + chunk_off(32 * warp + 2 * i + (lane >> 4), lane & 15, kPlane),
+                           kv_v + (int64_t)(rr[i] < 0 ? 0 : rr[i]) * kHd + (lane & 15) * 8, rr[i] < 0 ? 0u : 16u);
+            cp_async_arrive(&vfull[vs]);
+            e_cur = e_nxt;
+            d_cur = d_nxt;
+            e_nxt = e_far;
+        }
+        cp_async_wait_all();
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ MMA issuer
+        // S(u) is issued one tile ahead of P.V(u-1), so a tile's softmax runs
+        // while the previous tile's P.V is on the tensor core
+        if (lane == 0 && ntl > 0) {
+            const uint32_t fmt = F16 ? 0u : 1u;
+            const uint32_t idesc_s = make_idesc(fmt, fmt, M, kSlots);
+            const uint32_t idesc_pv = make_idesc(fmt, fmt, M, kHd) | (1u << 16);   // B (values) MN-major
+            auto issue_pv = [&](int u) {                 // O += P V of this CTA's tile u
+                const int vs = u % kVStages, pb = u & 1;
+                wait_phase(&pfull[pb], (u >> 1) & 1, a.status);
+                wait_phase(&vfull[vs], (u / kVStages) & 1, a.status);
+                fence_proxy_async_smem();        // copies landed by cp.async, read by the tensor core
+                tc_fence_after_sync();
+                const uint32_t vb = sbase + L::V + vs * kStageBytes;
+                const uint32_t pbase = sbase + L::P + pb * L::QPLANE;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_f16(tO, smem_desc_sw128(pbase + kk * 32),
+                            smem_desc_sw128_mn(vb + kk * 16 * 128, kPlane, 1024), idesc_pv,
+                            (u > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&vempty[vs]);
+                mma_commit(&pvdone[pb]);
+            };
+            for (int u = 0; u < ntl; ++u) {
+                const int ks = u % kKStages, sb = u & 1;
+                wait_phase(&kfull[ks], (u / kKStages) & 1, a.status);
+                wait_phase(&sfree[sb], ((u >> 1) & 1) ^ 1u, a.status);
+                fence_proxy_async_smem();
+                tc_fence_after_sync();
+                const uint32_t kb = sbase + L::K + ks * kStageBytes;
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_f16(tmem + sb * kSlots, smem_desc_sw128(sbase + L::Q + c * L::QPLANE + kk * 32),
+                                smem_desc_sw128(kb + c * kPlane + kk * 32), idesc_s, (c | kk) != 0);
+                mma_commit(&sfull[sb]);
+                mma_commit(&kempty[ks]);
+                if (u > 0) issue_pv(u - 1);
+            }
+            issue_pv(ntl - 1);
+        }
+    } else if constexpr (M == 64) {
+        // ------------------------------------------------------------ softmax (M = 64)
+        // Quarter q's 16 heads sit in lanes 32q..32q+15; read with the
+        // 16-lane shape, thread t holds heads 16q + t/4 and 16q + t/4 + 8 and,
+        // of each 8-key group j, keys 8j + 2(t%4) and 8j + 2(t%4) + 1; the four
+        // threads of a head combine their max and sum with two shuffles.
+        const int quarter = warp & 3;
+        const uint32_t tlane = (uint32_t)(quarter * 32) << 16;
+        const int t0 = lane & 3, t1 = lane >> 2;
+        const int hd[2] = {quarter * 16 + t1, quarter * 16 + t1 + 8};
+        float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+        for (int u = 0; u < ntl; ++u) {
+            const int ks = u % kKStages, sb = u & 1;
+            wait_phase(&sfull[sb], (u >> 1) & 1, a.status);
+            tc_fence_after_sync();
+            uint32_t sv[32];
+            tmem_ld_16x256b_x8(tmem + sb * kSlots + tlane, sv);
+            tmem_ld_wait();
+            // the stage's mask: its key stage cannot be refilled before these
+            // warps release it, so this phase is the current one
+            wait_phase(&kfull[ks], (u / kKStages) & 1, a.status);
+            const uint32_t mk0 = sMask[ks * 2], mk1 = sMask[ks * 2 + 1];
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&sfree[sb]);              // S buffer read
+                mbar_arrive(&kempty[ks]);             // mask read
+            }
             float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
+            for (int j = 0; j < 8; ++j)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const bool ok = (valid >> (nt * 8 + 2 * c + (e & 1))) & 1u;
-                    s[nt][e] = ok ? s[nt][e] * a.scale_log2 : -INFINITY;
-                    mx[e >> 1] = fmaxf(mx[e >> 1], s[nt][e]);
+                    const int key = 8 * j + 2 * t0 + (e & 1);
+                    const bool ok = ((key < 32 ? mk0 : mk1) >> (key & 31)) & 1u;
+                    const float x = ok ? __uint_as_float(sv[4 * j + e]) * a.scale_log2 : -INFINITY;
+                    sv[4 * j + e] = __float_as_uint(x);
+                    mx[e >> 1] = fmaxf(mx[e >> 1], x);
                 }
-            float base_[2], alpha[2];
+            float alpha[2], mb[2];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
-                mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
-                const float mn = fmaxf(m[h], mx[h]);
-                base_[h] = mn == -INFINITY ? 0.f : mn;
-                alpha[h] = exp2f(m[h] - base_[h]);
-                m[h] = mn;
+            for (int g = 0; g < 2; ++g) {
+                mx[g] = fmaxf(mx[g], __shfl_xor_sync(0xffffffffu, mx[g], 1));
+                mx[g] = fmaxf(mx[g], __shfl_xor_sync(0xffffffffu, mx[g], 2));
+                // move the running max only when this tile beats it by more than 2^8
+                alpha[g] = 1.f;
+                if (mx[g] > m_run[g] + kRescaleLog2 || (m_run[g] == -INFINITY && mx[g] > -INFINITY)) {
+                    alpha[g] = m_run[g] == -INFINITY ? 0.f : ex2(m_run[g] - mx[g]);
+                    m_run[g] = mx[g];
+                }
+                mb[g] = m_run[g] == -INFINITY ? 0.f : m_run[g];
             }
-            // the weights, rounded to dtype as the P.V product sees them, packed
-            // straight into A fragments; the normaliser sums the same values
+            uint32_t pk[16];                      // [j][head]: keys 8j+2t0, +1
             float rs[2] = {0.f, 0.f};
-            uint32_t pk[8][2];
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
+            for (int j = 0; j < 8; ++j)
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    pk[nt][h] = pack2<F16>(exp2f(s[nt][2 * h] - base_[h]), exp2f(s[nt][2 * h + 1] - base_[h]));
-                    rs[h] += unpack_lo<F16>(pk[nt][h]) + unpack_hi<F16>(pk[nt][h]);
+                for (int g = 0; g < 2; ++g) {
+                    const uint32_t w = pack2<F16>(ex2(__uint_as_float(sv[4 * j + 2 * g]) - mb[g]),
+                                                  ex2(__uint_as_float(sv[4 * j + 2 * g + 1]) - mb[g]));
+                    pk[2 * j + g] = w;
+                    rs[g] += unpack_lo<F16>(w) + unpack_hi<F16>(w);
                 }
 #pragma unroll
-            for (int h = 0; h < 2; ++h) l[h] = l[h] * alpha[h] + rs[h];
-            // the running max moved for some head of this warp: rescale O
-            if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
-#pragma unroll
-                for (int dn = 0; dn < 16; ++dn) {
-                    o[dn][0] *= alpha[0];
-                    o[dn][1] *= alpha[0];
-                    o[dn][2] *= alpha[1];
-                    o[dn][3] *= alpha[1];
-                }
+            for (int g = 0; g < 2; ++g) {
+                rs[g] += __shfl_xor_sync(0xffffffffu, rs[g], 1);
+                rs[g] += __shfl_xor_sync(0xffffffffu, rs[g], 2);
+                l_run[g] = l_run[g] * alpha[g] + rs[g];
             }
-            // O += P V
+            // the weights buffer of this tile was last read by P.V(u-2)
+            const int pb = u & 1;
+            if (u > 1) {
+                wait_phase(&pvdone[pb], ((u - 2) >> 1) & 1, a.status);
+                tc_fence_after_sync();
+            }
+            uint8_t *pbuf = base + L::P + pb * L::QPLANE;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint32_t pa[4] = {pk[2 * j][0], pk[2 * j][1], pk[2 * j + 1][0], pk[2 * j + 1][1]};
+            for (int j = 0; j < 8; ++j)
 #pragma unroll
-                for (int dp = 0; dp < 8; ++dp) {
-                    const int key = j * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
-                    const int ch = dp * 2 + (lane >> 4);
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4_t(vb + tile_off(key, ch), b0, b1, b2, b3);
-                    mma16816<F16>(o[2 * dp], pa, b0, b1);
-                    mma16816<F16>(o[2 * dp + 1], pa, b2, b3);
+                for (int g = 0; g < 2; ++g)
+                    *reinterpret_cast<uint32_t *>(pbuf + hd[g] * 128 + ((j ^ (hd[g] & 7)) << 4) + 4 * t0) = pk[2 * j + g];
+            // O *= alpha where some head of this warp moved its max (O holds the
+            // previous tiles once P.V(u-1) is done; the first tile's P.V
+            // overwrites it)
+            if (u > 0 && __any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
+                wait_phase(&pvdone[pb ^ 1], ((u - 1) >> 1) & 1, a.status);
+                tc_fence_after_sync();
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t o[32];
+                    tmem_ld_16x256b_x8(tO + tlane + 64 * c, o);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha[(e >> 1) & 1]);
+                    tmem_st_16x256b_x8(tO + tlane + 64 * c, o);
+                }
+                tmem_st_wait();
+            }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pfull[pb]);
+        }
+        if (ntl > 0) {
+            // the last P.V (its buffer's latest phase; waiting on a phase that
+            // has already completed returns at once)
+            wait_phase(&pvdone[(ntl - 1) & 1], ((ntl - 1) >> 1) & 1, a.status);
+            tc_fence_after_sync();
+        }
+        // ---- normalise and store (zeros and -inf when nothing was selected)
+        const float ln2 = 0.69314718055994531f;
+        float *sO = reinterpret_cast<float *>(base + L::K);              // [M][128], unnormalised (C > 1)
+        float *sM = reinterpret_cast<float *>(base + L::MERGE);
+        float *sL = sM + 128;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            uint32_t o[32];                       // columns 64c + 8j + 2t0 (+1) of heads hd[0], hd[1]
+            if (ntl > 0) {
+                tmem_ld_16x256b_x8(tO + tlane + 64 * c, o);
+                tmem_ld_wait();
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+#pragma unroll
+                for (int g = 0; g < 2; ++g) {
+                    const int col = 64 * c + 8 * j + 2 * t0;
+                    const float o0 = ntl > 0 ? __uint_as_float(o[4 * j + 2 * g]) : 0.f;
+                    const float o1 = ntl > 0 ? __uint_as_float(o[4 * j + 2 * g + 1]) : 0.f;
+                    if constexpr (C == 1) {
+                        if (hd[g] < a.N1) {
+                            const float inv = l_run[g] > 0.f ? 1.f / l_run[g] : 0.f;
+                            *reinterpret_cast<uint32_t *>(a.out + ((int64_t)row * a.N1 + hd[g]) * kHd + col) =
+                                l_run[g] > 0.f ? pack2<F16>(o0 * inv, o1 * inv) : 0u;
+                        }
+                    } else {
+                        sO[hd[g] * kHd + col] = o0;
+                        sO[hd[g] * kHd + col + 1] = o1;
+                    }
+                }
+        }
+        if (t0 == 0) {
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+                if constexpr (C == 1) {
+                    if (a.lse && hd[g] < a.N1)
+                        a.lse[(int64_t)row * a.N1 + hd[g]] =
+                            l_run[g] > 0.f ? (m_run[g] + log2f(l_run[g])) * ln2 : -INFINITY;
+                } else {
+                    sM[hd[g]] = m_run[g];
+                    sL[hd[g]] = l_run[g];
                 }
             }
         }
-        __syncthreads();                       // the buffers of tile t are refilled next
-        any_cur = any_next;
+    } else {
+        // ------------------------------------------------------------ softmax (M = 128)
+        const int quarter = warp & 3;             // tensor-memory lane quarter of this warp
+        const uint32_t tlane = (uint32_t)(quarter * 32) << 16;
+        // this thread's head: M = 64 keeps rows 16q..16q+15 in lanes 32q..32q+15
+        // of quarter q, M = 128 row r in lane r
+        const int h = M == 64 ? (lane < 16 ? quarter * 16 + lane : -1) : quarter * 32 + lane;
+        float m_run = -INFINITY, l_run = 0.f;     // log2-domain running max and sum
+        for (int u = 0; u < ntl; ++u) {
+            const int ks = u % kKStages, sb = u & 1;
+            wait_phase(&sfull[sb], (u >> 1) & 1, a.status);
+            tc_fence_after_sync();
+            uint32_t sv[64];
+            const uint32_t ts = tmem + sb * kSlots + tlane;
+            tmem_ld16_into<0>(ts, sv);
+            tmem_ld16_into<1>(ts, sv);
+            tmem_ld16_into<2>(ts, sv);
+            tmem_ld16_into<3>(ts, sv);
+            tmem_ld_wait();
+            // the stage's mask: its key stage cannot be refilled before these
+            // warps release it, so this phase is the current one
+            wait_phase(&kfull[ks], (u / kKStages) & 1, a.status);
+            const uint32_t mk0 = sMask[ks * 2], mk1 = sMask[ks * 2 + 1];
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&sfree[sb]);              // S buffer read
+                mbar_arrive(&kempty[ks]);             // mask read
+            }
+            float mx[16];
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+                const bool ok = ((j < 32 ? mk0 : mk1) >> (j & 31)) & 1u;
+                const float x = ok ? __uint_as_float(sv[j]) * a.scale_log2 : -INFINITY;
+                sv[j] = __float_as_uint(x);
+                mx[j & 15] = (j < 16) ? x : fmaxf(mx[j & 15], x);
+            }
+#pragma unroll
+            for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+                for (int j = 0; j < w; ++j) mx[j] = fmaxf(mx[j], mx[j + w]);
+            const float mt = mx[0];
+            // move the running max only when this tile beats it by more than 2^8
+            float alpha = 1.f;
+            if (h >= 0 && (mt > m_run + kRescaleLog2 || (m_run == -INFINITY && mt > -INFINITY))) {
+                alpha = m_run == -INFINITY ? 0.f : ex2(m_run - mt);
+                m_run = mt;
+            }
+            const float mb = m_run == -INFINITY ? 0.f : m_run;
+            float rs[8];
+            uint32_t pk[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                pk[j] = pack2<F16>(ex2(__uint_as_float(sv[2 * j]) - mb), ex2(__uint_as_float(sv[2 * j + 1]) - mb));
+                const float pr = unpack_lo<F16>(pk[j]) + unpack_hi<F16>(pk[j]);
+                rs[j & 7] = (j < 8) ? pr : rs[j & 7] + pr;
+            }
+#pragma unroll
+            for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+                for (int j = 0; j < w; ++j) rs[j] += rs[j + w];
+            l_run = l_run * alpha + rs[0];
+            // the weights buffer of this tile was last read by P.V(u-2)
+            const int pb = u & 1;
+            if (u > 1) {
+                wait_phase(&pvdone[pb], ((u - 2) >> 1) & 1, a.status);
+                tc_fence_after_sync();
+            }
+            if (h >= 0) {
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    *reinterpret_cast<uint4 *>(base + L::P + pb * L::QPLANE + chunk_off(h, ch, L::QPLANE)) =
+                        make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+            }
+            // O *= alpha where some head of this warp moved its max (O holds the
+            // previous tiles once P.V(u-1) is done; the first tile's P.V
+            // overwrites it)
+            const bool rescale = u > 0 && __any_sync(0xffffffffu, alpha != 1.f);
+            if (rescale) {
+                wait_phase(&pvdone[pb ^ 1], ((u - 1) >> 1) & 1, a.status);
+                tc_fence_after_sync();
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t o16[16];
+                    tmem_ld16(tO + tlane + 16 * c, o16);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) o16[e] = __float_as_uint(__uint_as_float(o16[e]) * alpha);
+                    tmem_st16(tO + tlane + 16 * c, o16);
+                }
+                tmem_st_wait();
+            }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pfull[pb]);
+        }
+        if (ntl > 0) {
+            // the last P.V (its buffer's latest phase; waiting on a phase that
+            // has already completed returns at once)
+            wait_phase(&pvdone[(ntl - 1) & 1], ((ntl - 1) >> 1) & 1, a.status);
+            tc_fence_after_sync();
+        }
+        // ---- normalise and store (zeros and -inf when nothing was selected)
+        if constexpr (C == 1) {
+            const float ln2 = 0.69314718055994531f;
+            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            uint16_t *orow = a.out + ((int64_t)row * a.N1 + (h < 0 ? 0 : h)) * kHd;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint32_t o16[16];
+                if (ntl > 0) {
+                    tmem_ld16(tO + tlane + 16 * c, o16);
+                    tmem_ld_wait();
+                }
+                if (h >= 0 && h < a.N1) {
+                    uint32_t w8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        w8[e] = ntl > 0 && l_run > 0.f
+                                    ? pack2<F16>(__uint_as_float(o16[2 * e]) * inv, __uint_as_float(o16[2 * e + 1]) * inv)
+                                    : 0u;
+                    *reinterpret_cast<uint4 *>(orow + 16 * c) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+                    *reinterpret_cast<uint4 *>(orow + 16 * c + 8) = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+                }
+            }
+            if (a.lse && h >= 0 && h < a.N1)
+                a.lse[(int64_t)row * a.N1 + h] = l_run > 0.f ? (m_run + log2f(l_run)) * ln2 : -INFINITY;
+        } else {
+            // partials into this CTA's shared memory (the key/value rings are
+            // free: every MMA has completed)
+            float *sO = reinterpret_cast<float *>(base + L::K);              // [M][128], unnormalised
+            float *sM = reinterpret_cast<float *>(base + L::MERGE);          // [128]
+            float *sL = sM + 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint32_t o16[16];
+                if (ntl > 0) {
+                    tmem_ld16(tO + tlane + 16 * c, o16);
+                    tmem_ld_wait();
+                }
+                if (h >= 0)
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) sO[h * kHd + 16 * c + e] = ntl > 0 ? __uint_as_float(o16[e]) : 0.f;
+            }
+            if (h >= 0) {
+                sM[h] = m_run;
+                sL[h] = l_run;
+            }
+        }
     }
 
-    // ---- normalise and store (zeros and -inf when nothing was selected)
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        l[h] += __shfl_xor_sync(0xffffffffu, l[h], 1);
-        l[h] += __shfl_xor_sync(0xffffffffu, l[h], 2);
-    }
     if constexpr (C > 1) {
-        // partials into this CTA's shared memory (the tile buffers are free)
-        float *sO = reinterpret_cast<float *>(base);                 // [N1][128], unnormalised
-        float *sM = reinterpret_cast<float *>(base + 4 * kTileBytes + kRowMapBytes);    // [N1]
-        float *sL = sM + 128;                                        // [N1]
-        const int h0 = warp * 16 + g, h1 = h0 + 8;
-#pragma unroll
-        for (int dn = 0; dn < 16; ++dn) {
-            const int d = dn * 8 + 2 * c;
-            sO[h0 * kHd + d] = o[dn][0];
-            sO[h0 * kHd + d + 1] = o[dn][1];
-            sO[h1 * kHd + d] = o[dn][2];
-            sO[h1 * kHd + d + 1] = o[dn][3];
-        }
-        if (c == 0) {
-            sM[h0] = m[0];
-            sL[h0] = l[0];
-            sM[h1] = m[1];
-            sL[h1] = l[1];
-        }
+        // CTA `part` merges heads [part*N1/C, (part+1)*N1/C) over the C partials
+        float *sO = reinterpret_cast<float *>(base + L::K);
+        float *sM = reinterpret_cast<float *>(base + L::MERGE);
+        float *sL = sM + 128;
         cooperative_groups::cluster_group cl = cooperative_groups::this_cluster();
         cl.sync();
-        // CTA `part` merges heads [part*N1/C, (part+1)*N1/C) over the C partials
-        const int hpc = a.N1 / C;
         const float ln2 = 0.69314718055994531f;
-        for (int e = tid; e < hpc * kHd; e += NT) {
-            const int h = part * hpc + e / kHd, d = e % kHd;
-            float M = -INFINITY;
+        const int hpc = a.N1 / C;
+        for (int e = tid; e < hpc * kHd; e += kThreads) {
+            const int hh = part * hpc + e / kHd, d = e % kHd;
+            float Mx = -INFINITY;
 #pragma unroll
-            for (int r = 0; r < C; ++r) M = fmaxf(M, cl.map_shared_rank(sM, r)[h]);
-            float L = 0.f, O = 0.f;
-            if (M != -INFINITY) {
+            for (int r = 0; r < C; ++r) Mx = fmaxf(Mx, cl.map_shared_rank(sM, r)[hh]);
+            float Ls = 0.f, Os = 0.f;
+            if (Mx != -INFINITY) {
 #pragma unroll
                 for (int r = 0; r < C; ++r) {
-                    const float mr = cl.map_shared_rank(sM, r)[h];
+                    const float mr = cl.map_shared_rank(sM, r)[hh];
                     if (mr == -INFINITY) continue;
-                    const float w = exp2f(mr - M);
-                    L += cl.map_shared_rank(sL, r)[h] * w;
-                    O += cl.map_shared_rank(sO, r)[h * kHd + d] * w;
+                    const float w = exp2f(mr - Mx);
+                    Ls += cl.map_shared_rank(sL, r)[hh] * w;
+                    Os += cl.map_shared_rank(sO, r)[hh * kHd + d] * w;
                 }
             }
-            const float v = L > 0.f ? O / L : 0.f;
-            a.out[((int64_t)row * a.N1 + h) * kHd + d] =
+            const float v = Ls > 0.f ? Os / Ls : 0.f;
+            a.out[((int64_t)row * a.N1 + hh) * kHd + d] =
                 F16 ? __half_as_ushort(__float2half_rn(v)) : __bfloat16_as_ushort(__float2bfloat16_rn(v));
-            if (d == 0 && a.lse) a.lse[(int64_t)row * a.N1 + h] = L > 0.f ? (M + log2f(L)) * ln2 : -INFINITY;
+            if (d == 0 && a.lse) a.lse[(int64_t)row * a.N1 + hh] = Ls > 0.f ? (Mx + log2f(Ls)) * ln2 : -INFINITY;
         }
         cl.sync();                             // every peer has read this CTA's partials
-        return;
     }
-    const float inv0 = l[0] > 0.f ? 1.f / l[0] : 0.f, inv1 = l[1] > 0.f ? 1.f / l[1] : 0.f;
-    uint16_t *orow = a.out + ((int64_t)row * a.N1 + warp * 16) * kHd;
-#pragma unroll
-    for (int dn = 0; dn < 16; ++dn) {
-        const int d = dn * 8 + 2 * c;
-        *reinterpret_cast<uint32_t *>(orow + g * kHd + d) = pack2<F16>(o[dn][0] * inv0, o[dn][1] * inv0);
-        *reinterpret_cast<uint32_t *>(orow + (g + 8) * kHd + d) = pack2<F16>(o[dn][2] * inv1, o[dn][3] * inv1);
-    }
-    if (a.lse && c == 0) {
-        const float ln2 = 0.69314718055994531f;
-        float *lr = a.lse + (int64_t)row * a.N1 + warp * 16;
-        lr[g] = l[0] > 0.f ? (m[0] + log2f(l[0])) * ln2 : -INFINITY;
-        lr[g + 8] = l[1] > 0.f ? (m[1] + log2f(l[1])) * ln2 : -INFINITY;
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    if (warp == 2) tmem_dealloc(tmem, 256);
+}
+
+// Rows when the key tensor is empty: out = 0, lse = -inf.
+template <bool F16>
+__global__ void sfa_empty_kernel(uint16_t *out, float *lse, int64_t rows, int N1)
+{
+    const int64_t n = rows * N1 * kHd;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+        out[e] = 0;
+        if (lse && e % kHd == 0) lse[e / kHd] = -INFINITY;
     }
 }
 
-template <int NW, bool F16, int C>
+template <int M, bool F16, int C>
 cudaError_t launch(const SfaArgs &a, int rows, cudaStream_t s)
 {
-    auto kern = sfa_kernel<NW, F16, C>;
-    cudaError_t e = li::set_max_dynamic_smem(reinterpret_cast<const void *>(kern), kSmem);
+    auto kern = sfa_kernel<M, F16, C>;
+    const int smem = Layout<M>::BYTES;
+    cudaError_t e = li::set_max_dynamic_smem(reinterpret_cast<const void *>(kern), smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)rows * C);
-    cfg.blockDim = dim3(32 * NW);
-    cfg.dynamicSmemBytes = kSmem;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -454,37 +807,31 @@ cudaError_t launch(const SfaArgs &a, int rows, cudaStream_t s)
     return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-template <int NW, bool F16>
+template <int M, bool F16>
 cudaError_t launch_split(const SfaArgs &a, int rows, int split, cudaStream_t s)
 {
     switch (split) {
-    case 1: return launch<NW, F16, 1>(a, rows, s);
-    case 2: return launch<NW, F16, 2>(a, rows, s);
-    case 4: return launch<NW, F16, 4>(a, rows, s);
-    case 8: return launch<NW, F16, 8>(a, rows, s);
+    case 1: return launch<M, F16, 1>(a, rows, s);
+    case 2: return launch<M, F16, 2>(a, rows, s);
+    case 4: return launch<M, F16, 4>(a, rows, s);
+    case 8: return launch<M, F16, 8>(a, rows, s);
     }
     return cudaErrorInvalidValue;
 }
 
 template <bool F16>
-cudaError_t launch_nw(const SfaArgs &a, int rows, int split, cudaStream_t s)
+cudaError_t launch_m(const SfaArgs &a, int rows, int split, cudaStream_t s)
 {
-    switch (a.N1) {
-    case 16: return launch_split<1, F16>(a, rows, split, s);
-    case 32: return launch_split<2, F16>(a, rows, split, s);
-    case 64: return launch_split<4, F16>(a, rows, split, s);
-    case 128: return launch_split<8, F16>(a, rows, split, s);
-    }
-    return cudaErrorInvalidValue;
+    return a.N1 <= 64 ? launch_split<64, F16>(a, rows, split, s) : launch_split<128, F16>(a, rows, split, s);
 }
 
 // CTAs per row: enough to give every SM two rows' worth of work when rows are
-// few (decode), at least one 64-key tile per CTA, a power of two up to 8.
+// few (decode), at least two 64-key tiles per CTA, a power of two up to 8.
 int choose_split(int64_t rows, int K, int sms)
 {
-    const int ntiles = (K + kTile - 1) / kTile;
+    const int ntiles = (K + kSlots - 1) / kSlots;
     int c = 1;
-    while (c < kMaxSplit && rows * c < 2LL * sms && 2 * c <= ntiles) c *= 2;
+    while (c < kMaxSplit && rows * c < 2LL * sms && 4 * c <= ntiles) c *= 2;
     return c;
 }
 
@@ -575,9 +922,19 @@ extern "C" LI_API li_status li_sparse_attention(const li_sfa_params *p, const vo
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int split = choose_split(rows, a.K, sms);
-    const cudaError_t e = p->dtype == LI_FP16 ? launch_nw<true>(a, (int)rows, split, s)
-                                              : launch_nw<false>(a, (int)rows, split, s);
+    cudaError_t e;
+    if (key_rows == 0) {
+        // no key can be selected: every row is empty
+        const int grid = (int)((rows * p->N1 * kHd + 255) / 256 < 4096 ? (rows * p->N1 * kHd + 255) / 256 : 4096);
+        if (p->dtype == LI_FP16)
+            sfa_empty_kernel<true><<<grid, 256, 0, s>>>(a.out, a.lse, rows, p->N1);
+        else
+            sfa_empty_kernel<false><<<grid, 256, 0, s>>>(a.out, a.lse, rows, p->N1);
+        e = cudaGetLastError();
+    } else {
+        const int split = choose_split(rows, a.K, sms);
+        e = p->dtype == LI_FP16 ? launch_m<true>(a, (int)rows, split, s) : launch_m<false>(a, (int)rows, split, s);
+    }
     if (e != cudaSuccess) {
         char msg[200];
         snprintf(msg, sizeof msg, "li_sparse_attention: launch failed (%s)", cudaGetErrorString(e));

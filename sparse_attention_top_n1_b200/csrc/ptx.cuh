@@ -255,6 +255,39 @@ __device__ __forceinline__ void tmem_ld_wait16(uint32_t (&r)[16])
 }
 
 
+// 32 lanes x 16 columns of 32-bit data from registers into TMEM (one column
+// per register); complete with tmem_st_wait before the data is read.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait()
+{
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor for an MN-major operand stored with the
+// 128-byte swizzle: along MN, 64 16-bit elements (128 B) per swizzle row and
+// `lbo_bytes` between consecutive 64-element groups; along K, one 128-byte row
+// per K index, 8-row atoms of 1024 B, `sbo_bytes` between consecutive atoms.
+__device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t saddr, uint32_t lbo_bytes,
+                                                       uint32_t sbo_bytes)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
 // Shared-memory matrix descriptor for a K-major operand stored with the
 // 128-byte swizzle (rows of 128 B, 8-row atoms of 1024 B).  Fields: start
 // address >> 4 in bits [0,14), leading byte offset >> 4 in [16,30) (unused for

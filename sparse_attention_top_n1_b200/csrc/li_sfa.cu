@@ -210,6 +210,35 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
+// max of three (one instruction on sm_100)
+__device__ __forceinline__ float fmax3(float x, float y, float z)
+{
+    float m;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(x), "f"(y), "f"(z));
+    return m;
+}
+
+// (d0, d1) = (a0 * b0 + c0, a1 * b1 + c1) as one packed fp32 instruction
+__device__ __forceinline__ void ffma2(float &d0, float &d1, float a0, float a1, float b0, float b1, float c0,
+                                      float c1)
+{
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+// (d0, d1) += (x0, x1) as one packed fp32 instruction
+__device__ __forceinline__ void fadd2(float &d0, float &d1, float x0, float x1)
+{
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%0, %1};\n\tmov.b64 rb, {%2, %3};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(x0), "f"(x1));
+}
+
 // Bounded wait on an mbarrier phase; an expired wait flags LI_DEV_TIMEOUT and
 // the caller goes on (results are then undefined; the context stays usable).
 __device__ __forceinline__ void wait_phase(uint64_t *bar, uint32_t parity, int32_t *status)
@@ -459,46 +488,57 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
                 mbar_arrive(&sfree[sb]);              // S buffer read
                 mbar_arrive(&kempty[ks]);             // mask read
             }
-            float mx[2] = {-INFINITY, -INFINITY};
+            // empty slots get a raw score of -inf (a tile with every slot
+            // filled skips the test); the scale is positive, so the max is
+            // taken on raw scores and scaled once
+            if ((mk0 & mk1) != 0xffffffffu) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
+                for (int j = 0; j < 8; ++j)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int key = 8 * j + 2 * t0 + (e & 1);
-                    const bool ok = ((key < 32 ? mk0 : mk1) >> (key & 31)) & 1u;
-                    const float x = ok ? __uint_as_float(sv[4 * j + e]) * a.scale_log2 : -INFINITY;
-                    sv[4 * j + e] = __float_as_uint(x);
-                    mx[e >> 1] = fmaxf(mx[e >> 1], x);
-                }
-            float alpha[2], mb[2];
+                    for (int e = 0; e < 4; ++e) {
+                        const int key = 8 * j + 2 * t0 + (e & 1);
+                        if (!(((key < 32 ? mk0 : mk1) >> (key & 31)) & 1u)) sv[4 * j + e] = 0xff800000u;
+                    }
+            }
+            float mx[2], alpha[2], mb[2];
 #pragma unroll
             for (int g = 0; g < 2; ++g) {
+                auto s_ = [&](int k) { return __uint_as_float(sv[4 * (k >> 1) + 2 * g + (k & 1)]); };
+                const float a0 = fmax3(s_(0), s_(1), s_(2)), a1 = fmax3(s_(3), s_(4), s_(5));
+                const float a2 = fmax3(s_(6), s_(7), s_(8)), a3 = fmax3(s_(9), s_(10), s_(11));
+                const float a4 = fmax3(s_(12), s_(13), s_(14));
+                mx[g] = fmaxf(fmax3(a0, a1, a2), fmax3(a3, a4, s_(15)));
                 mx[g] = fmaxf(mx[g], __shfl_xor_sync(0xffffffffu, mx[g], 1));
                 mx[g] = fmaxf(mx[g], __shfl_xor_sync(0xffffffffu, mx[g], 2));
+                mx[g] *= a.scale_log2;
                 // move the running max only when this tile beats it by more than 2^8
                 alpha[g] = 1.f;
                 if (mx[g] > m_run[g] + kRescaleLog2 || (m_run[g] == -INFINITY && mx[g] > -INFINITY)) {
                     alpha[g] = m_run[g] == -INFINITY ? 0.f : ex2(m_run[g] - mx[g]);
                     m_run[g] = mx[g];
                 }
-                mb[g] = m_run[g] == -INFINITY ? 0.f : m_run[g];
+                mb[g] = m_run[g] == -INFINITY ? 0.f : -m_run[g];
             }
+            // weights exp2(scale_log2 * s - m), two keys per packed fma
             uint32_t pk[16];                      // [j][head]: keys 8j+2t0, +1
-            float rs[2] = {0.f, 0.f};
+            float rs[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
             for (int j = 0; j < 8; ++j)
 #pragma unroll
                 for (int g = 0; g < 2; ++g) {
-                    const uint32_t w = pack2<F16>(ex2(__uint_as_float(sv[4 * j + 2 * g]) - mb[g]),
-                                                  ex2(__uint_as_float(sv[4 * j + 2 * g + 1]) - mb[g]));
+                    float x0, x1;
+                    ffma2(x0, x1, __uint_as_float(sv[4 * j + 2 * g]), __uint_as_float(sv[4 * j + 2 * g + 1]),
+                          a.scale_log2, a.scale_log2, mb[g], mb[g]);
+                    const uint32_t w = pack2<F16>(ex2(x0), ex2(x1));
                     pk[2 * j + g] = w;
-                    rs[g] += unpack_lo<F16>(w) + unpack_hi<F16>(w);
+                    fadd2(rs[g][0], rs[g][1], unpack_lo<F16>(w), unpack_hi<F16>(w));
                 }
 #pragma unroll
             for (int g = 0; g < 2; ++g) {
-                rs[g] += __shfl_xor_sync(0xffffffffu, rs[g], 1);
-                rs[g] += __shfl_xor_sync(0xffffffffu, rs[g], 2);
-                l_run[g] = l_run[g] * alpha[g] + rs[g];
+                float r = rs[g][0] + rs[g][1];
+                r += __shfl_xor_sync(0xffffffffu, r, 1);
+                r += __shfl_xor_sync(0xffffffffu, r, 2);
+                l_run[g] = l_run[g] * alpha[g] + r;
             }
             // the weights buffer of this tile was last read by P.V(u-2)
             const int pb = u & 1;
@@ -613,39 +653,41 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
                 mbar_arrive(&sfree[sb]);              // S buffer read
                 mbar_arrive(&kempty[ks]);             // mask read
             }
-            float mx[16];
+            if ((mk0 & mk1) != 0xffffffffu) {     // empty slots: raw score -inf
 #pragma unroll
-            for (int j = 0; j < 64; ++j) {
-                const bool ok = ((j < 32 ? mk0 : mk1) >> (j & 31)) & 1u;
-                const float x = ok ? __uint_as_float(sv[j]) * a.scale_log2 : -INFINITY;
-                sv[j] = __float_as_uint(x);
-                mx[j & 15] = (j < 16) ? x : fmaxf(mx[j & 15], x);
+                for (int j = 0; j < 64; ++j)
+                    if (!(((j < 32 ? mk0 : mk1) >> (j & 31)) & 1u)) sv[j] = 0xff800000u;
             }
+            float mx[22];
 #pragma unroll
-            for (int w = 8; w > 0; w >>= 1)
+            for (int j = 0; j < 21; ++j)
+                mx[j] = fmax3(__uint_as_float(sv[3 * j]), __uint_as_float(sv[3 * j + 1]), __uint_as_float(sv[3 * j + 2]));
+            mx[21] = __uint_as_float(sv[63]);
 #pragma unroll
-                for (int j = 0; j < w; ++j) mx[j] = fmaxf(mx[j], mx[j + w]);
-            const float mt = mx[0];
+            for (int j = 0; j < 7; ++j) mx[j] = fmax3(mx[3 * j], mx[3 * j + 1], mx[3 * j + 2]);
+            const float mt = fmaxf(fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5])),
+                                   fmaxf(mx[6], mx[21])) * a.scale_log2;
             // move the running max only when this tile beats it by more than 2^8
             float alpha = 1.f;
             if (h >= 0 && (mt > m_run + kRescaleLog2 || (m_run == -INFINITY && mt > -INFINITY))) {
                 alpha = m_run == -INFINITY ? 0.f : ex2(m_run - mt);
                 m_run = mt;
             }
-            const float mb = m_run == -INFINITY ? 0.f : m_run;
-            float rs[8];
+            const float mb = m_run == -INFINITY ? 0.f : -m_run;
+            float rs[4][2] = {};
             uint32_t pk[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                pk[j] = pack2<F16>(ex2(__uint_as_float(sv[2 * j]) - mb), ex2(__uint_as_float(sv[2 * j + 1]) - mb));
-                const float pr = unpack_lo<F16>(pk[j]) + unpack_hi<F16>(pk[j]);
-                rs[j & 7] = (j < 8) ? pr : rs[j & 7] + pr;
+                float x0, x1;
+                ffma2(x0, x1, __uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1]), a.scale_log2, a.scale_log2,
+                      mb, mb);
+                pk[j] = pack2<F16>(ex2(x0), ex2(x1));
+                fadd2(rs[j & 3][0], rs[j & 3][1], unpack_lo<F16>(pk[j]), unpack_hi<F16>(pk[j]));
             }
-#pragma unroll
-            for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-                for (int j = 0; j < w; ++j) rs[j] += rs[j + w];
-            l_run = l_run * alpha + rs[0];
+            rs[0][0] += rs[2][0] + (rs[1][0] + rs[3][0]);
+            rs[0][1] += rs[2][1] + (rs[1][1] + rs[3][1]);
+            rs[0][0] += rs[0][1];
+            l_run = l_run * alpha + rs[0][0];
             // the weights buffer of this tile was last read by P.V(u-2)
             const int pb = u & 1;
             if (u > 1) {

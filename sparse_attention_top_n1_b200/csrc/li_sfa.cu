@@ -67,7 +67,8 @@ constexpr int kHd = 128;                  // D = Dv
 constexpr int kSlots = 64;                // selected keys per tile: the N of S, the K of P.V
 constexpr int kThreads = 224;             // two producer warps, MMA issuer, four softmax warps
 constexpr int kProducers = 64;            // one producer thread per slot of a tile
-constexpr int kKStages = 2, kVStages = 2;
+constexpr int kKStages = 3, kVStages = 2;
+constexpr int kMaskRing = 8;             // slot-validity masks in flight (>= kKStages + 2)
 constexpr int kStageBytes = kSlots * kHd * 2;   // one key or value tile: two 64-column planes
 constexpr int kPlane = kSlots * 128;            // one 64-column plane of a tile
 constexpr int kMaxSplit = 8;              // CTAs (one cluster) sharing a row's keys
@@ -96,13 +97,13 @@ struct Layout {
     static constexpr int Q = 0;                             // [2][M][128 B]
     static constexpr int K = Q + 2 * QPLANE;                // [kKStages][2][64][128 B]
     static constexpr int V = K + kKStages * kStageBytes;    // [kVStages][2][64][128 B]
-    static constexpr int P = V + kVStages * kStageBytes;    // [2][M][128 B]: weights, 64 keys along K
-    static constexpr int MASK = P + 2 * QPLANE;             // uint32 [kKStages][2]
-    static constexpr int BARS = MASK + 32;                  // mbarriers
-    static constexpr int NBARS = 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 2;
+    static constexpr int P = V + kVStages * kStageBytes;    // [M][128 B]: weights, 64 keys along K
+    static constexpr int MASK = P + QPLANE;                 // uint32 [kMaskRing][2]
+    static constexpr int BARS = MASK + kMaskRing * 8;       // mbarriers
+    static constexpr int NBARS = 2 * kKStages + 2 * kVStages + 2 + 2 + 1 + 1 + kMaskRing;
     static constexpr int TSLOT = BARS + NBARS * 8;
-    static constexpr int MERGE = TSLOT + 16;                // float [2][128]: a cluster's (m, l)
-    static constexpr int END = MERGE + 2 * 128 * 4;
+    static constexpr int MERGE = TSLOT + 16;                // float [3][128]: a cluster's (m, l), merge weights
+    static constexpr int END = MERGE + 3 * 128 * 4;
     static constexpr int BYTES = END + 1024;                // + alignment of the base
 };
 
@@ -270,7 +271,8 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
     uint64_t *kfull = bars, *kempty = bars + kKStages;
     uint64_t *vfull = bars + 2 * kKStages, *vempty = vfull + kVStages;
     uint64_t *sfull = vempty + kVStages, *sfree = sfull + 2;
-    uint64_t *pfull = sfree + 2, *pvdone = pfull + 2;     // per weights buffer
+    uint64_t *pfull = sfree + 2, *pvdone = pfull + 1;     // the weights buffer
+    uint64_t *mfull = pvdone + 1;                         // [kMaskRing]
     uint32_t *tslot = reinterpret_cast<uint32_t *>(base + L::TSLOT);
     const uint32_t sbase = smem_u32(base);
 
@@ -316,8 +318,8 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
 
     if (tid == 0) {
         for (int s = 0; s < kKStages; ++s) {
-            mbar_init(&kfull[s], kProducers + 2); // every producer thread's copies, the two mask words
-            mbar_init(&kempty[s], 1 + 4);         // the S commit and the four softmax warps
+            mbar_init(&kfull[s], kProducers);     // every producer thread's copies
+            mbar_init(&kempty[s], 1);             // the S commit
         }
         for (int s = 0; s < kVStages; ++s) {
             mbar_init(&vfull[s], kProducers);     // every producer thread's copies
@@ -327,10 +329,9 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
             mbar_init(&sfull[s], 1);
             mbar_init(&sfree[s], 4);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&pfull[s], 4);
-            mbar_init(&pvdone[s], 1);
-        }
+        mbar_init(pfull, 4);                      // the four softmax warps
+        mbar_init(pvdone, 1);                     // the P.V commit
+        for (int s = 0; s < kMaskRing; ++s) mbar_init(&mfull[s], 2);   // lane 0 of each producer warp
         fence_mbarrier_init();
     }
     if (warp == 2) tmem_alloc(tslot, 256);        // S: two buffers of 64 columns; O: 128-255
@@ -392,11 +393,15 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
 #pragma unroll
             for (int i = 0; i < 16; ++i) rr[i] = __shfl_sync(0xffffffffu, r, 2 * i + (lane >> 4));
             const int ks = u % kKStages, vs = u % kVStages;
-            // keys of tile u and its validity mask (read by the softmax warps after kfull)
+            // keys of tile u
             wait_phase(&kempty[ks], ((u / kKStages) & 1) ^ 1u, a.status);
+            // its validity mask: ring entry u % kMaskRing was last read by the
+            // softmax of tile u - kMaskRing, which released its S buffer
+            // before S(u - kMaskRing + 2) was issued, which precedes the
+            // release of this key stage (kMaskRing >= kKStages + 2)
             if (lane == 0) {
-                sMask[ks * 2 + warp] = ok;
-                mbar_arrive(&kfull[ks]);
+                sMask[(u % kMaskRing) * 2 + warp] = ok;
+                mbar_arrive(&mfull[u % kMaskRing]);
             }
             const uint32_t kd = sbase + L::K + ks * kStageBytes;
 #pragma unroll
@@ -426,20 +431,20 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
             const uint32_t idesc_s = make_idesc(fmt, fmt, M, kSlots);
             const uint32_t idesc_pv = make_idesc(fmt, fmt, M, kHd) | (1u << 16);   // B (values) MN-major
             auto issue_pv = [&](int u) {                 // O += P V of this CTA's tile u
-                const int vs = u % kVStages, pb = u & 1;
-                wait_phase(&pfull[pb], (u >> 1) & 1, a.status);
+                const int vs = u % kVStages;
+                wait_phase(pfull, u & 1, a.status);
                 wait_phase(&vfull[vs], (u / kVStages) & 1, a.status);
                 fence_proxy_async_smem();        // copies landed by cp.async, read by the tensor core
                 tc_fence_after_sync();
                 const uint32_t vb = sbase + L::V + vs * kStageBytes;
-                const uint32_t pbase = sbase + L::P + pb * L::QPLANE;
+                const uint32_t pbase = sbase + L::P;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_f16(tO, smem_desc_sw128(pbase + kk * 32),
                             smem_desc_sw128_mn(vb + kk * 16 * 128, kPlane, 1024), idesc_pv,
                             (u > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&vempty[vs]);
-                mma_commit(&pvdone[pb]);
+                mma_commit(pvdone);
             };
             for (int u = 0; u < ntl; ++u) {
                 const int ks = u % kKStages, sb = u & 1;
@@ -472,22 +477,17 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
         const int hd[2] = {quarter * 16 + t1, quarter * 16 + t1 + 8};
         float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
         for (int u = 0; u < ntl; ++u) {
-            const int ks = u % kKStages, sb = u & 1;
+            const int sb = u & 1;
             wait_phase(&sfull[sb], (u >> 1) & 1, a.status);
             tc_fence_after_sync();
             uint32_t sv[32];
             tmem_ld_16x256b_x8(tmem + sb * kSlots + tlane, sv);
             tmem_ld_wait();
-            // the stage's mask: its key stage cannot be refilled before these
-            // warps release it, so this phase is the current one
-            wait_phase(&kfull[ks], (u / kKStages) & 1, a.status);
-            const uint32_t mk0 = sMask[ks * 2], mk1 = sMask[ks * 2 + 1];
+            wait_phase(&mfull[u % kMaskRing], (u / kMaskRing) & 1, a.status);
+            const uint32_t mk0 = sMask[(u % kMaskRing) * 2], mk1 = sMask[(u % kMaskRing) * 2 + 1];
             tc_fence_before_sync();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&sfree[sb]);              // S buffer read
-                mbar_arrive(&kempty[ks]);             // mask read
-            }
+            if (lane == 0) mbar_arrive(&sfree[sb]);   // S buffer (and mask entry) read
             // empty slots get a raw score of -inf (a tile with every slot
             // filled skips the test); the scale is positive, so the max is
             // taken on raw scores and scaled once
@@ -540,13 +540,13 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
                 r += __shfl_xor_sync(0xffffffffu, r, 2);
                 l_run[g] = l_run[g] * alpha[g] + r;
             }
-            // the weights buffer of this tile was last read by P.V(u-2)
-            const int pb = u & 1;
-            if (u > 1) {
-                wait_phase(&pvdone[pb], ((u - 2) >> 1) & 1, a.status);
+            // the weights buffer was last read by P.V(u-1), which also
+            // completes O for the rescale below
+            if (u > 0) {
+                wait_phase(pvdone, (u - 1) & 1, a.status);
                 tc_fence_after_sync();
             }
-            uint8_t *pbuf = base + L::P + pb * L::QPLANE;
+            uint8_t *pbuf = base + L::P;
 #pragma unroll
             for (int j = 0; j < 8; ++j)
 #pragma unroll
@@ -556,8 +556,6 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
             // previous tiles once P.V(u-1) is done; the first tile's P.V
             // overwrites it)
             if (u > 0 && __any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
-                wait_phase(&pvdone[pb ^ 1], ((u - 1) >> 1) & 1, a.status);
-                tc_fence_after_sync();
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     uint32_t o[32];
@@ -572,12 +570,12 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
             fence_proxy_async_smem();
             tc_fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&pfull[pb]);
+            if (lane == 0) mbar_arrive(pfull);
         }
         if (ntl > 0) {
             // the last P.V (its buffer's latest phase; waiting on a phase that
             // has already completed returns at once)
-            wait_phase(&pvdone[(ntl - 1) & 1], ((ntl - 1) >> 1) & 1, a.status);
+            wait_phase(pvdone, (ntl - 1) & 1, a.status);
             tc_fence_after_sync();
         }
         // ---- normalise and store (zeros and -inf when nothing was selected)
@@ -633,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
         const int h = M == 64 ? (lane < 16 ? quarter * 16 + lane : -1) : quarter * 32 + lane;
         float m_run = -INFINITY, l_run = 0.f;     // log2-domain running max and sum
         for (int u = 0; u < ntl; ++u) {
-            const int ks = u % kKStages, sb = u & 1;
+            const int sb = u & 1;
             wait_phase(&sfull[sb], (u >> 1) & 1, a.status);
             tc_fence_after_sync();
             uint32_t sv[64];
@@ -643,16 +641,11 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
             tmem_ld16_into<2>(ts, sv);
             tmem_ld16_into<3>(ts, sv);
             tmem_ld_wait();
-            // the stage's mask: its key stage cannot be refilled before these
-            // warps release it, so this phase is the current one
-            wait_phase(&kfull[ks], (u / kKStages) & 1, a.status);
-            const uint32_t mk0 = sMask[ks * 2], mk1 = sMask[ks * 2 + 1];
+            wait_phase(&mfull[u % kMaskRing], (u / kMaskRing) & 1, a.status);
+            const uint32_t mk0 = sMask[(u % kMaskRing) * 2], mk1 = sMask[(u % kMaskRing) * 2 + 1];
             tc_fence_before_sync();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&sfree[sb]);              // S buffer read
-                mbar_arrive(&kempty[ks]);             // mask read
-            }
+            if (lane == 0) mbar_arrive(&sfree[sb]);   // S buffer (and mask entry) read
             if ((mk0 & mk1) != 0xffffffffu) {     // empty slots: raw score -inf
 #pragma unroll
                 for (int j = 0; j < 64; ++j)
@@ -688,16 +681,16 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
             rs[0][1] += rs[2][1] + (rs[1][1] + rs[3][1]);
             rs[0][0] += rs[0][1];
             l_run = l_run * alpha + rs[0][0];
-            // the weights buffer of this tile was last read by P.V(u-2)
-            const int pb = u & 1;
-            if (u > 1) {
-                wait_phase(&pvdone[pb], ((u - 2) >> 1) & 1, a.status);
+            // the weights buffer was last read by P.V(u-1), which also
+            // completes O for the rescale below
+            if (u > 0) {
+                wait_phase(pvdone, (u - 1) & 1, a.status);
                 tc_fence_after_sync();
             }
             if (h >= 0) {
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch)
-                    *reinterpret_cast<uint4 *>(base + L::P + pb * L::QPLANE + chunk_off(h, ch, L::QPLANE)) =
+                    *reinterpret_cast<uint4 *>(base + L::P + chunk_off(h, ch, L::QPLANE)) =
                         make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
             }
             // O *= alpha where some head of this warp moved its max (O holds the
@@ -705,8 +698,6 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
             // overwrites it)
             const bool rescale = u > 0 && __any_sync(0xffffffffu, alpha != 1.f);
             if (rescale) {
-                wait_phase(&pvdone[pb ^ 1], ((u - 1) >> 1) & 1, a.status);
-                tc_fence_after_sync();
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     uint32_t o16[16];
@@ -721,12 +712,12 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
             fence_proxy_async_smem();
             tc_fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&pfull[pb]);
+            if (lane == 0) mbar_arrive(pfull);
         }
         if (ntl > 0) {
             // the last P.V (its buffer's latest phase; waiting on a phase that
             // has already completed returns at once)
-            wait_phase(&pvdone[(ntl - 1) & 1], ((ntl - 1) >> 1) & 1, a.status);
+            wait_phase(pvdone, (ntl - 1) & 1, a.status);
             tc_fence_after_sync();
         }
         // ---- normalise and store (zeros and -inf when nothing was selected)
@@ -783,30 +774,48 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
         float *sO = reinterpret_cast<float *>(base + L::K);
         float *sM = reinterpret_cast<float *>(base + L::MERGE);
         float *sL = sM + 128;
+        float *sWt = sL + 128;                 // [hpc][C]: each partial's weight exp2(m_r - M) / L
         cooperative_groups::cluster_group cl = cooperative_groups::this_cluster();
         cl.sync();
         const float ln2 = 0.69314718055994531f;
         const int hpc = a.N1 / C;
-        for (int e = tid; e < hpc * kHd; e += kThreads) {
-            const int hh = part * hpc + e / kHd, d = e % kHd;
+        // per (head, partial): the merged max and normaliser, then the weight
+        // of that partial's unnormalised output
+        for (int e = tid; e < hpc * C; e += kThreads) {
+            const int hl = e / C, r = e % C, hh = part * hpc + hl;
             float Mx = -INFINITY;
 #pragma unroll
-            for (int r = 0; r < C; ++r) Mx = fmaxf(Mx, cl.map_shared_rank(sM, r)[hh]);
-            float Ls = 0.f, Os = 0.f;
+            for (int q = 0; q < C; ++q) Mx = fmaxf(Mx, cl.map_shared_rank(sM, q)[hh]);
+            float Ls = 0.f;
             if (Mx != -INFINITY) {
 #pragma unroll
-                for (int r = 0; r < C; ++r) {
-                    const float mr = cl.map_shared_rank(sM, r)[hh];
-                    if (mr == -INFINITY) continue;
-                    const float w = exp2f(mr - Mx);
-                    Ls += cl.map_shared_rank(sL, r)[hh] * w;
-                    Os += cl.map_shared_rank(sO, r)[hh * kHd + d] * w;
+                for (int q = 0; q < C; ++q) {
+                    const float mq = cl.map_shared_rank(sM, q)[hh];
+                    if (mq != -INFINITY) Ls += cl.map_shared_rank(sL, q)[hh] * exp2f(mq - Mx);
                 }
             }
-            const float v = Ls > 0.f ? Os / Ls : 0.f;
-            a.out[((int64_t)row * a.N1 + hh) * kHd + d] =
-                F16 ? __half_as_ushort(__float2half_rn(v)) : __bfloat16_as_ushort(__float2bfloat16_rn(v));
-            if (d == 0 && a.lse) a.lse[(int64_t)row * a.N1 + hh] = Ls > 0.f ? (Mx + log2f(Ls)) * ln2 : -INFINITY;
+            const float mr = cl.map_shared_rank(sM, r)[hh];
+            sWt[e] = (Ls > 0.f && mr != -INFINITY) ? exp2f(mr - Mx) / Ls : 0.f;
+            if (r == 0 && a.lse) a.lse[(int64_t)row * a.N1 + hh] = Ls > 0.f ? (Mx + log2f(Ls)) * ln2 : -INFINITY;
+        }
+        __syncthreads();
+        // out = sum_r weight_r * O_r, four columns per thread and step
+        for (int e = tid; e < hpc * (kHd / 4); e += kThreads) {
+            const int hl = e / (kHd / 4), d4 = e % (kHd / 4), hh = part * hpc + hl;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int r = 0; r < C; ++r) {
+                const float w = sWt[hl * C + r];
+                if (w != 0.f) {
+                    const float4 o = reinterpret_cast<const float4 *>(cl.map_shared_rank(sO, r))[hh * (kHd / 4) + d4];
+                    acc.x += w * o.x;
+                    acc.y += w * o.y;
+                    acc.z += w * o.z;
+                    acc.w += w * o.w;
+                }
+            }
+            *reinterpret_cast<uint2 *>(a.out + ((int64_t)row * a.N1 + hh) * kHd + 4 * d4) =
+                make_uint2(pack2<F16>(acc.x, acc.y), pack2<F16>(acc.z, acc.w));
         }
         cl.sync();                             // every peer has read this CTA's partials
     }
@@ -867,13 +876,14 @@ cudaError_t launch_m(const SfaArgs &a, int rows, int split, cudaStream_t s)
     return a.N1 <= 64 ? launch_split<64, F16>(a, rows, split, s) : launch_split<128, F16>(a, rows, split, s);
 }
 
-// CTAs per row: enough to give every SM two rows' worth of work when rows are
-// few (decode), at least two 64-key tiles per CTA, a power of two up to 8.
+// CTAs per row when rows are few (decode): the largest power of two up to 8
+// that keeps the grid within one wave of two CTAs per SM, with at least four
+// 64-key tiles per CTA.
 int choose_split(int64_t rows, int K, int sms)
 {
     const int ntiles = (K + kSlots - 1) / kSlots;
     int c = 1;
-    while (c < kMaxSplit && rows * c < 2LL * sms && 4 * c <= ntiles) c *= 2;
+    while (c < kMaxSplit && rows * c * 2 <= 2LL * sms && 4 * c * 2 <= ntiles) c *= 2;
     return c;
 }
 

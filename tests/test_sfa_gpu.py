@@ -74,6 +74,12 @@ CASES = {
     "k1": dict(seed=35, B=1, S1=20, S2=50, N1=64, K=1),
     "k64_noncausal_scale": dict(seed=36, B=2, S1=12, S2=80, N1=32, K=64, causal=False, softmax_scale=0.3),
     "big_scale": dict(seed=37, B=1, S1=16, S2=128, N1=16, K=64, causal=False, softmax_scale=4.0),
+    # few rows: each row's keys are split over a cluster of 2, 4 or 8 CTAs
+    "split2_bsnd": dict(seed=41, B=2, S1=3, S2=1500, N1=32, K=600, causal=False),
+    "split4_pa_n128": dict(seed=42, layout_kv="PA_BSND", B=3, S1=2, k_lens=[1500, 2000, 900], N1=128,
+                           K=1100, block_size=64),
+    "split8_pa_decode": dict(seed=43, layout_kv="PA_BSND", B=4, S1=1, k_lens=[3000, 5000, 2500, 4100], N1=64,
+                             K=2048, block_size=128, holes=0.1),
 }
 
 

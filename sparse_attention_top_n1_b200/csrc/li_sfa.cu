@@ -335,20 +335,61 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
         fence_mbarrier_init();
     }
     if (warp == 2) tmem_alloc(tslot, 256);        // S: two buffers of 64 columns; O: 128-255
-    // Q into shared memory (heads beyond N1 are zero rows)
-    for (int e = tid; e < M * 16; e += kThreads) {
-        const int r = e >> 4, ch = e & 15;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (r < a.N1 && valid_row) v = *reinterpret_cast<const uint4 *>(a.q + ((int64_t)row * a.N1 + r) * kHd + ch * 8);
-        *reinterpret_cast<uint4 *>(base + L::Q + chunk_off(r, ch, L::QPLANE)) = v;
+    // the producers' slot resolution (thread p of warps 0-1 owns slot p); the
+    // first tiles' index loads, and the first block-table load, are issued
+    // around the query load so their latencies overlap it
+    const int32_t *irow = a.idx + (int64_t)row * a.K;
+    const int sp = tid;                           // slot of this thread
+    const bool pa = a.layout_kv == LI_PA_BSND;
+    const int64_t bt_row = (int64_t)b * a.max_blocks_per_seq;
+    auto load_idx = [&](int t) -> int {           // index of this slot in tile t (or -1)
+        const int j = t * kSlots + sp;
+        return (t < t_end && j < a.K) ? irow[j] : -1;
+    };
+    auto load_blk = [&](int e) -> int {           // block id behind a valid index
+        return (pa && e >= 0 && e < Sk) ? a.block_table[bt_row + e / a.block_size] : 0;
+    };
+    auto row_of = [&](int e, int id) -> int {     // key row, or -1 (flags bad entries)
+        if (e >= 0 && e < Sk) {
+            if (!pa) return (int)(k_off + e);
+            if (id >= 0 && id < a.num_blocks) return id * a.block_size + e % a.block_size;
+            if (a.status) atomicOr(a.status, LI_DEV_BAD_BLOCK);
+            return -1;
+        }
+        if (e != -1 && a.status) atomicOr(a.status, LI_DEV_BAD_INDEX);
+        return -1;
+    };
+    int e_cur = -1, e_nxt = -1, d_cur = 0;
+    if (warp < 2) {
+        e_cur = load_idx(t_begin);
+        e_nxt = load_idx(t_begin + 1);
     }
+    // Q into shared memory (heads beyond N1 are zero rows): every load of
+    // this thread is issued before the first store, so the query costs one
+    // memory latency
+    {
+        constexpr int kQIter = (M * 16 + kThreads - 1) / kThreads;
+        uint4 qv[kQIter];
+#pragma unroll
+        for (int k = 0; k < kQIter; ++k) {
+            const int e = tid + k * kThreads, r = e >> 4, ch = e & 15;
+            qv[k] = make_uint4(0, 0, 0, 0);
+            if (e < M * 16 && r < a.N1 && valid_row)
+                qv[k] = *reinterpret_cast<const uint4 *>(a.q + ((int64_t)row * a.N1 + r) * kHd + ch * 8);
+        }
+#pragma unroll
+        for (int k = 0; k < kQIter; ++k) {
+            const int e = tid + k * kThreads, r = e >> 4, ch = e & 15;
+            if (e < M * 16) *reinterpret_cast<uint4 *>(base + L::Q + chunk_off(r, ch, L::QPLANE)) = qv[k];
+        }
+    }
+    if (warp < 2) d_cur = load_blk(e_cur);
     fence_proxy_async_smem();
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tslot;
     const uint32_t tO = tmem + 128;
-    const int32_t *irow = a.idx + (int64_t)row * a.K;
     const uint16_t *kv_k = a.k, *kv_v = a.v;
 
     if (warp < 2) {
@@ -361,28 +402,6 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
         // slot.  Each stage is signalled by the copies themselves: the
         // thread's arrival on the stage's full barrier is deferred by the
         // copy unit until all its earlier copies have landed.
-        const int sp = tid;                      // slot of this thread
-        const bool pa = a.layout_kv == LI_PA_BSND;
-        const int64_t bt_row = (int64_t)b * a.max_blocks_per_seq;
-        auto load_idx = [&](int t) -> int {      // index of this slot in tile t (or -1)
-            const int j = t * kSlots + sp;
-            return (t < t_end && j < a.K) ? irow[j] : -1;
-        };
-        auto load_blk = [&](int e) -> int {      // block id behind a valid index
-            return (pa && e >= 0 && e < Sk) ? a.block_table[bt_row + e / a.block_size] : 0;
-        };
-        auto row_of = [&](int e, int id) -> int {  // key row, or -1 (flags bad entries)
-            if (e >= 0 && e < Sk) {
-                if (!pa) return (int)(k_off + e);
-                if (id >= 0 && id < a.num_blocks) return id * a.block_size + e % a.block_size;
-                if (a.status) atomicOr(a.status, LI_DEV_BAD_BLOCK);
-                return -1;
-            }
-            if (e != -1 && a.status) atomicOr(a.status, LI_DEV_BAD_INDEX);
-            return -1;
-        };
-        int e_cur = load_idx(t_begin), e_nxt = load_idx(t_begin + 1);
-        int d_cur = load_blk(e_cur);
         for (int u = 0; u < ntl; ++u) {
             const int t = t_begin + u;
             const int r = row_of(e_cur, d_cur);

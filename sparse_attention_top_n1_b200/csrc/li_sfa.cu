@@ -85,6 +85,7 @@ struct SfaArgs {
     int32_t B, S1, S2, T1, T2, N1, K;
     int32_t num_blocks, block_size, max_blocks_per_seq;
     float scale_log2;                     // softmax scale * log2(e)
+    int32_t bs_shift;                     // log2(block_size), or -1
 };
 
 // Shared memory of one CTA (byte offsets from a 1024-byte aligned base).  Q,
@@ -347,12 +348,13 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
         return (t < t_end && j < a.K) ? irow[j] : -1;
     };
     auto load_blk = [&](int e) -> int {           // block id behind a valid index
-        return (pa && e >= 0 && e < Sk) ? a.block_table[bt_row + e / a.block_size] : 0;
+        return (pa && e >= 0 && e < Sk) ? a.block_table[bt_row + (a.bs_shift >= 0 ? e >> a.bs_shift : e / a.block_size)] : 0;
     };
     auto row_of = [&](int e, int id) -> int {     // key row, or -1 (flags bad entries)
         if (e >= 0 && e < Sk) {
             if (!pa) return (int)(k_off + e);
-            if (id >= 0 && id < a.num_blocks) return id * a.block_size + e % a.block_size;
+            if (id >= 0 && id < a.num_blocks)
+                return id * a.block_size + (a.bs_shift >= 0 ? e & (a.block_size - 1) : e % a.block_size);
             if (a.status) atomicOr(a.status, LI_DEV_BAD_BLOCK);
             return -1;
         }
@@ -990,6 +992,11 @@ extern "C" LI_API li_status li_sparse_attention(const li_sfa_params *p, const vo
     a.block_size = p->block_size;
     a.max_blocks_per_seq = p->max_blocks_per_seq;
     a.scale_log2 = p->softmax_scale * 1.4426950408889634f;
+    a.bs_shift = -1;
+    if (p->block_size > 0 && (p->block_size & (p->block_size - 1)) == 0) {
+        a.bs_shift = 0;
+        while ((1 << a.bs_shift) < p->block_size) ++a.bs_shift;
+    }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

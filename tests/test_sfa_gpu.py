@@ -80,6 +80,11 @@ CASES = {
                            K=1100, block_size=64),
     "split8_pa_decode": dict(seed=43, layout_kv="PA_BSND", B=4, S1=1, k_lens=[3000, 5000, 2500, 4100], N1=64,
                              K=2048, block_size=128, holes=0.1),
+    "split8_n16_bsnd": dict(seed=44, B=2, S1=1, S2=3000, N1=16, K=2048, causal=False),
+    "split4_tnd_pa_fp16": dict(seed=45, layout_q="TND", layout_kv="PA_BSND", dtype="fp16", B=3, q_lens=[1, 2, 1],
+                               k_lens=[3000, 1500, 2200], N1=32, K=1200, block_size=32),
+    "pa_block_not_pow2": dict(seed=46, layout_kv="PA_BSND", B=2, S1=3, k_lens=[700, 450], N1=64, K=300,
+                              block_size=48),
 }
 
 

@@ -102,7 +102,7 @@ struct Layout {
     static constexpr int MASK = P + QPLANE;                 // uint32 [kMaskRing][2]
     static constexpr int BARS = MASK + kMaskRing * 8;       // mbarriers
     static constexpr int NBARS = 2 * kKStages + 2 * kVStages + 2 + 2 + 1 + 1 + kMaskRing;
-    static constexpr int TSLOT = BARS + NBARS * 8;
+    static constexpr int TSLOT = BARS + NBARS * 8;         // TMEM address, then the abort flag
     static constexpr int MERGE = TSLOT + 16;                // float [3][128]: a cluster's (m, l), merge weights
     static constexpr int END = MERGE + 3 * 128 * 4;
     static constexpr int BYTES = END + 1024;                // + alignment of the base
@@ -241,16 +241,27 @@ __device__ __forceinline__ void fadd2(float &d0, float &d1, float x0, float x1)
         : "f"(x0), "f"(x1));
 }
 
-// Bounded wait on an mbarrier phase; an expired wait flags LI_DEV_TIMEOUT and
-// the caller goes on (results are then undefined; the context stays usable).
-__device__ __forceinline__ void wait_phase(uint64_t *bar, uint32_t parity, int32_t *status)
+// Bounded wait on an mbarrier phase.  A wait that expires (2 s) flags
+// LI_DEV_TIMEOUT and sets the CTA's abort flag; from then on every wait of
+// the CTA returns after one suspended try (at most about a microsecond), and
+// so does a wait of another CTA once it sees the flag in `status`, so a
+// broken pipeline ends the kernel promptly (results are then undefined; the
+// context stays usable).
+__device__ __forceinline__ void wait_phase(uint64_t *bar, uint32_t parity, int32_t *status, volatile int *abort)
 {
     // the waiting thread is suspended in hardware (up to 1 us per try) until
     // the phase completes, instead of spinning on the issue slots
     if (mbar_try_wait(bar, parity)) return;
     const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait_sleep(bar, parity, 1000u)) {
+    for (uint32_t it = 1; !mbar_try_wait_sleep(bar, parity, 1000u); ++it) {
+        if (*abort) return;
+        // another CTA's timeout, looked at every 256 tries (a global load)
+        if ((it & 255u) == 0 && status && (*reinterpret_cast<volatile int32_t *>(status) & LI_DEV_TIMEOUT)) {
+            *abort = 1;
+            return;
+        }
         if ((int64_t)(global_timer_ns() - t0) > 2000000000LL) {
+            *abort = 1;
             if (status) atomicOr(status, LI_DEV_TIMEOUT);
             return;
         }
@@ -275,6 +286,7 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
     uint64_t *pfull = sfree + 2, *pvdone = pfull + 1;     // the weights buffer
     uint64_t *mfull = pvdone + 1;                         // [kMaskRing]
     uint32_t *tslot = reinterpret_cast<uint32_t *>(base + L::TSLOT);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(base + L::TSLOT + 4);
     const uint32_t sbase = smem_u32(base);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -333,6 +345,7 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
         mbar_init(pfull, 4);                      // the four softmax warps
         mbar_init(pvdone, 1);                     // the P.V commit
         for (int s = 0; s < kMaskRing; ++s) mbar_init(&mfull[s], 2);   // lane 0 of each producer warp
+        *abort_flag = 0;
         fence_mbarrier_init();
     }
     if (warp == 2) tmem_alloc(tslot, 256);        // S: two buffers of 64 columns; O: 128-255
@@ -415,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
             for (int i = 0; i < 16; ++i) rr[i] = __shfl_sync(0xffffffffu, r, 2 * i + (lane >> 4));
             const int ks = u % kKStages, vs = u % kVStages;
             // keys of tile u
-            wait_phase(&kempty[ks], ((u / kKStages) & 1) ^ 1u, a.status);
+            wait_phase(&kempty[ks], ((u / kKStages) & 1) ^ 1u, a.status, abort_flag);
             // its validity mask: ring entry u % kMaskRing was last read by the
             // softmax of tile u - kMaskRing, which released its S buffer
             // before S(u - kMaskRing + 2) was issued, which precedes the
@@ -431,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
                            kv_k + (int64_t)(rr[i] < 0 ? 0 : rr[i]) * kHd + (lane & 15) * 8, rr[i] < 0 ? 0u : 16u);
             cp_async_arrive(&kfull[ks]);
             // values of tile u
-            wait_phase(&vempty[vs], ((u / kVStages) & 1) ^ 1u, a.status);
+            wait_phase(&vempty[vs], ((u / kVStages) & 1) ^ 1u, a.status, abort_flag);
             const uint32_t vd = sbase + L::V + vs * kStageBytes;
 #pragma unroll
             for (int i = 0; i < 16; ++i)
@@ -453,8 +466,8 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
             const uint32_t idesc_pv = make_idesc(fmt, fmt, M, kHd) | (1u << 16);   // B (values) MN-major
             auto issue_pv = [&](int u) {                 // O += P V of this CTA's tile u
                 const int vs = u % kVStages;
-                wait_phase(pfull, u & 1, a.status);
-                wait_phase(&vfull[vs], (u / kVStages) & 1, a.status);
+                wait_phase(pfull, u & 1, a.status, abort_flag);
+                wait_phase(&vfull[vs], (u / kVStages) & 1, a.status, abort_flag);
                 fence_proxy_async_smem();        // copies landed by cp.async, read by the tensor core
                 tc_fence_after_sync();
                 const uint32_t vb = sbase + L::V + vs * kStageBytes;
@@ -469,8 +482,8 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
             };
             for (int u = 0; u < ntl; ++u) {
                 const int ks = u % kKStages, sb = u & 1;
-                wait_phase(&kfull[ks], (u / kKStages) & 1, a.status);
-                wait_phase(&sfree[sb], ((u >> 1) & 1) ^ 1u, a.status);
+                wait_phase(&kfull[ks], (u / kKStages) & 1, a.status, abort_flag);
+                wait_phase(&sfree[sb], ((u >> 1) & 1) ^ 1u, a.status, abort_flag);
                 fence_proxy_async_smem();
                 tc_fence_after_sync();
                 const uint32_t kb = sbase + L::K + ks * kStageBytes;
@@ -499,12 +512,12 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
         float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
         for (int u = 0; u < ntl; ++u) {
             const int sb = u & 1;
-            wait_phase(&sfull[sb], (u >> 1) & 1, a.status);
+            wait_phase(&sfull[sb], (u >> 1) & 1, a.status, abort_flag);
             tc_fence_after_sync();
             uint32_t sv[32];
             tmem_ld_16x256b_x8(tmem + sb * kSlots + tlane, sv);
             tmem_ld_wait();
-            wait_phase(&mfull[u % kMaskRing], (u / kMaskRing) & 1, a.status);
+            wait_phase(&mfull[u % kMaskRing], (u / kMaskRing) & 1, a.status, abort_flag);
             const uint32_t mk0 = sMask[(u % kMaskRing) * 2], mk1 = sMask[(u % kMaskRing) * 2 + 1];
             tc_fence_before_sync();
             __syncwarp();
@@ -564,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
             // the weights buffer was last read by P.V(u-1), which also
             // completes O for the rescale below
             if (u > 0) {
-                wait_phase(pvdone, (u - 1) & 1, a.status);
+                wait_phase(pvdone, (u - 1) & 1, a.status, abort_flag);
                 tc_fence_after_sync();
             }
             uint8_t *pbuf = base + L::P;
@@ -596,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
         if (ntl > 0) {
             // the last P.V (its buffer's latest phase; waiting on a phase that
             // has already completed returns at once)
-            wait_phase(pvdone, (ntl - 1) & 1, a.status);
+            wait_phase(pvdone, (ntl - 1) & 1, a.status, abort_flag);
             tc_fence_after_sync();
         }
         // ---- normalise and store (zeros and -inf when nothing was selected)
@@ -653,7 +666,7 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
         float m_run = -INFINITY, l_run = 0.f;     // log2-domain running max and sum
         for (int u = 0; u < ntl; ++u) {
             const int sb = u & 1;
-            wait_phase(&sfull[sb], (u >> 1) & 1, a.status);
+            wait_phase(&sfull[sb], (u >> 1) & 1, a.status, abort_flag);
             tc_fence_after_sync();
             uint32_t sv[64];
             const uint32_t ts = tmem + sb * kSlots + tlane;
@@ -662,7 +675,7 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
             tmem_ld16_into<2>(ts, sv);
             tmem_ld16_into<3>(ts, sv);
             tmem_ld_wait();
-            wait_phase(&mfull[u % kMaskRing], (u / kMaskRing) & 1, a.status);
+            wait_phase(&mfull[u % kMaskRing], (u / kMaskRing) & 1, a.status, abort_flag);
             const uint32_t mk0 = sMask[(u % kMaskRing) * 2], mk1 = sMask[(u % kMaskRing) * 2 + 1];
             tc_fence_before_sync();
             __syncwarp();
@@ -705,7 +718,7 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
             // the weights buffer was last read by P.V(u-1), which also
             // completes O for the rescale below
             if (u > 0) {
-                wait_phase(pvdone, (u - 1) & 1, a.status);
+                wait_phase(pvdone, (u - 1) & 1, a.status, abort_flag);
                 tc_fence_after_sync();
             }
             if (h >= 0) {
@@ -738,7 +751,7 @@ __global__ void __launch_bounds__(kThreads, M == 64 ? 2 : 1) sfa_kernel(const Sf
         if (ntl > 0) {
             // the last P.V (its buffer's latest phase; waiting on a phase that
             // has already completed returns at once)
-            wait_phase(pvdone, (ntl - 1) & 1, a.status);
+            wait_phase(pvdone, (ntl - 1) & 1, a.status, abort_flag);
             tc_fence_after_sync();
         }
         // ---- normalise and store (zeros and -inf when nothing was selected)

@@ -17,11 +17,11 @@
 //              table for a paged pool; an empty or invalid slot becomes a
 //              masked zero row) and gather the 64 key rows and 64 value rows
 //              with 16-byte cp.async copies, one 256-byte row per half warp
-//              and instruction, into two-stage key and value rings in the
-//              128-byte-swizzled layout the tensor core reads; each thread's
-//              arrival on a stage's full barrier is deferred by the copy unit
-//              until its copies have landed; the tile's slot-validity mask
-//              travels with its key stage;
+//              and instruction, into a three-stage key ring and a two-stage
+//              value ring in the 128-byte-swizzled layout the tensor core
+//              reads; each thread's arrival on a stage's full barrier is
+//              deferred by the copy unit until its copies have landed; the
+//              tile's slot-validity mask goes to a ring of its own;
 //   warp 2     issues S = Q K^T on tcgen05.mma (M = the heads, 64 or 128
 //              rows with zero rows for N1 < 64; N = 64 keys; K = D = 128)
 //              into one of two tensor-memory buffers, one tile ahead of
@@ -32,13 +32,13 @@
 //              (M = 64: four threads per head with the 16-lane load shape,
 //              combined by two shuffles; M = 128: one thread per head), scales
 //              the logits into the log2 domain, masks empty slots, rounds the
-//              weights exp2(s - m) to the input type and writes them to a
-//              double-buffered shared-memory tile (the normaliser sums the
-//              same rounded values, so the output stays a convex combination
-//              of values); the running max m moves only when a tile's max
-//              beats it by more than 2^8, and only then is O rescaled in
-//              tensor memory, so the weights stay below 256 and O is touched
-//              rarely.
+//              weights exp2(s - m) to the input type and writes them to the
+//              shared-memory weights tile once the previous P V has read it
+//              (the normaliser sums the same rounded values, so the output
+//              stays a convex combination of values); the running max m
+//              moves only when a tile's max beats it by more than 2^8, and
+//              only then is O rescaled in tensor memory, so the weights stay
+//              below 256 and O is touched rarely.
 // out = O / l and lse = ln 2 * (m + log2 l) are written once per row.
 #include <cuda.h>
 #include <cuda_bf16.h>

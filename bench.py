@@ -299,6 +299,10 @@ class ClockSampler:
 
 
 def dist_setup():
+    """Rank, world size and this rank's GPU.  The process group carries only
+    the barriers and the max of the timings: NCCL by default; LI_BENCH_BACKEND
+    =gloo runs it on the host, which lets several ranks share a GPU (their
+    kernels never wait on one another) to exercise the sharded path."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -307,17 +311,21 @@ def dist_setup():
 
         import torch
         import torch.distributed as dist
+        local = local % max(1, torch.cuda.device_count())
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist.init_process_group(os.environ.get("LI_BENCH_BACKEND", "nccl"),
+                                timeout=datetime.timedelta(seconds=120))
     return ws, rank, local
 
 
-def allreduce_max(x, device="cuda"):
+def allreduce_max(x, device=None):
     """Max of a host float over all ranks (timing only; no data-path use)."""
     import torch
     import torch.distributed as dist
     if not dist.is_initialized():
         return x
+    if device is None:
+        device = "cpu" if dist.get_backend() == "gloo" else "cuda"
     t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())

@@ -256,9 +256,16 @@ LI_API li_status li_indexer_noalloc(const li_params *p, const void *query, const
  *   out            [rows, N1, Dv] in dtype (device)
  *   lse            fp32 [rows, N1] (device) or NULL
  *   status         device int32 that receives LI_DEV_* bits by atomic OR, or
- *                  NULL; the caller clears it
+ *                  NULL; the caller clears it.  LI_DEV_BAD_INDEX: an entry
+ *                  outside [-1, Sk_b) (skipped); LI_DEV_BAD_BLOCK: a
+ *                  block_table entry outside [0, num_blocks) behind a valid
+ *                  index (skipped); LI_DEV_TIMEOUT: a pipeline wait expired
+ *                  (out and lse are then undefined; the kernel still ends)
+ * Pointers: query, key, value and out 16-byte aligned; sparse_indices, lse and
+ * status 4-byte aligned (else LI_ERR_SHAPE, nothing launched).
  * Accumulation is fp32 on the tensor cores; the softmax weights enter the P.V
- * product rounded to dtype.  Needs no workspace.  One launch.
+ * product rounded to dtype.  Needs no workspace.  One launch (a thread-block
+ * cluster per row when rows are few).
  */
 #define LI_DEV_BAD_INDEX     0x20  /* sparse attention: an index outside [-1, Sk) (skipped) */
 typedef struct {

@@ -17,7 +17,7 @@
 //              table for a paged pool; an empty or invalid slot becomes a
 //              masked zero row) and gather the 64 key rows and 64 value rows
 //              with 16-byte cp.async copies, one 256-byte row per half warp
-//              and instruction, into a three-stage key ring and a two-stage
+//              and instruction, into a two-stage key ring and a three-stage
 //              value ring in the 128-byte-swizzled layout the tensor core
 //              reads; each thread's arrival on a stage's full barrier is
 //              deferred by the copy unit until its copies have landed; the
@@ -67,7 +67,7 @@ constexpr int kHd = 128;                  // D = Dv
 constexpr int kSlots = 64;                // selected keys per tile: the N of S, the K of P.V
 constexpr int kThreads = 224;             // two producer warps, MMA issuer, four softmax warps
 constexpr int kProducers = 64;            // one producer thread per slot of a tile
-constexpr int kKStages = 3, kVStages = 2;
+constexpr int kKStages = 2, kVStages = 3;
 constexpr int kMaskRing = 8;             // slot-validity masks in flight (>= kKStages + 2)
 constexpr int kStageBytes = kSlots * kHd * 2;   // one key or value tile: two 64-column planes
 constexpr int kPlane = kSlots * 128;            // one 64-column plane of a tile

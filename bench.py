@@ -504,6 +504,105 @@ class Calls:
         return f
 
 
+def e2e_pieces(p):
+    """Row pieces for the end-to-end leg: one per 4096 query rows, up to 8."""
+    return max(1, min(8, p.rows // 4096))
+
+
+def time_e2e_pipelined(li, p, inp, calls, dev, npieces, steps, warmup, flush_l2):
+    """End to end with host buffers, the transfers overlapped with the work:
+    the query rows are split into `npieces` contiguous, pair-balanced pieces
+    (the same row split as the multi-GPU path), each its own li_indexer /
+    li_quant_indexer call.  One stream copies the key-side inputs and then
+    each piece's query-side inputs host -> device, one runs the calls in
+    order as their inputs land, one copies each piece's output rows back as
+    it completes; the timed region runs from the first copy to the last.
+    Every byte a call reads is copied every step.  The pieces' outputs are
+    checked bit for bit against the whole-problem call's."""
+    import dataclasses
+
+    import torch
+
+    from sparse_attention_top_n1_b200 import shard
+    aq, ak, cr = inp.get("act_q"), inp.get("act_k"), inp.get("cmp_residual_k")
+    cost = shard.row_costs(p, aq, ak, cr)
+    plan = [pc for r0, r1 in shard.split_rows(cost, npieces) for pc in shard.pieces_for_range(p, r0, r1, aq, ak, cr)]
+    d = calls.d
+    pin = lambda t: t.contiguous().pin_memory()
+    # key-side tensors, whole, once per step (pieces share them)
+    key_side = [k for k in ("key", "k_scale", "block_table") if d.get(k) is not None]
+    shared = [(pin(inp[k]), d[k]) for k in key_side]
+    pieces = []
+    for pc in plan:
+        sp = dataclasses.replace(p, **pc.fields)
+        dev_in = shard.piece_inputs(pc, p, d, lambda a: torch.from_numpy(a).to(dev))
+        host_in = shard.piece_inputs(pc, p, inp)
+        copies = [(pin(host_in[k]), dev_in[k]) for k in dev_in if k not in key_side]
+        pr = li.make_params(sp)
+        if dev_in.get("cmp_residual_k") is not None:
+            pr.cmp_residual_k = dev_in["cmp_residual_k"].data_ptr()
+        wsb = li.alloc_workspace(pr, dev)
+        oi = calls.idx[pc.r0:pc.r1]
+        ov = calls.val[pc.r0:pc.r1] if calls.val is not None else None
+        hi = torch.empty(oi.shape, dtype=oi.dtype).pin_memory()
+        hv = torch.empty(ov.shape, dtype=ov.dtype).pin_memory() if ov is not None else None
+        pieces.append((pr, dev_in, copies, wsb, oi, ov, hi, hv))
+    # the whole-problem call's result (the last timed call left it here): the
+    # pieces must reproduce it bit for bit
+    ref_i = calls.idx.clone()
+    ref_v = calls.val.clone() if calls.val is not None else None
+    h2d = sum(h.numel() * h.element_size() for h, _ in shared)
+    h2d += sum(h.numel() * h.element_size() for pc in pieces for h, _ in pc[2])
+    d2h = p.rows * p.sparse_count * (4 + 4 * p.return_value)
+    s_in, s_run, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    main = torch.cuda.current_stream(dev)
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    st, en = [mk() for _ in range(steps + warmup)], [mk() for _ in range(steps + warmup)]
+    for s_ in range(steps + warmup):
+        flush_l2()
+        st[s_].record(main)
+        for x in (s_in, s_run, s_out):
+            x.wait_stream(main)
+        with torch.cuda.stream(s_in):
+            for h, dv in shared:
+                dv.copy_(h, non_blocking=True)
+        for pr, dev_in, copies, wsb, oi, ov, hi, hv in pieces:
+            with torch.cuda.stream(s_in):
+                for h, dv in copies:
+                    dv.copy_(h, non_blocking=True)
+            landed = s_in.record_event()
+            s_run.wait_event(landed)
+            with torch.cuda.stream(s_run):
+                if p.quant:
+                    li.li_quant_indexer(pr, dev_in["query"], dev_in["key"], dev_in["weights"], dev_in.get("q_scale"),
+                                        dev_in.get("k_scale"), dev_in.get("act_q"), dev_in.get("act_k"),
+                                        dev_in.get("block_table"), oi, ov, wsb)
+                else:
+                    li.li_indexer(pr, dev_in["query"], dev_in["key"], dev_in["weights"], dev_in.get("act_q"),
+                                  dev_in.get("act_k"), dev_in.get("block_table"), oi, ov, wsb)
+            done = s_run.record_event()
+            s_out.wait_event(done)
+            with torch.cuda.stream(s_out):
+                hi.copy_(oi, non_blocking=True)
+                if hv is not None:
+                    hv.copy_(ov, non_blocking=True)
+        main.wait_stream(s_out)
+        main.wait_stream(s_run)
+        en[s_].record(main)
+    torch.cuda.synchronize()
+    for pr, dev_in, copies, wsb, oi, ov, hi, hv in pieces:
+        f = li.li_read_device_status(wsb)
+        if f:
+            raise SystemExit("end-to-end piece: device status 0x%x" % f)
+    if not torch.equal(calls.idx, ref_i) or (ref_v is not None and not torch.equal(
+            calls.val.view(torch.int32), ref_v.view(torch.int32))):
+        raise SystemExit("end-to-end pieces differ from the whole-problem call")
+    e_ms = sum(st[s_].elapsed_time(en[s_]) for s_ in range(warmup, steps + warmup))
+    return {"value": p.rows * steps / (e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "pieces": len(pieces),
+            "overlap": "host->device copies, the calls and device->host copies on three streams, by row piece"}
+
+
 def time_indexer(name, args, ctx, steps, warmup, cpu_budget, with_e2e=True):
     """Time `steps` calls of workload `name` on this rank; returns the record."""
     import torch
@@ -611,7 +710,10 @@ def time_indexer(name, args, ctx, steps, warmup, cpu_budget, with_e2e=True):
     # end to end through the C ABI with host buffers: H2D of this rank's inputs
     # from pinned memory, the call, D2H of its output rows, all timed
     e2e = None
-    if with_e2e and not (args.no_e2e or args.plain):
+    npieces = e2e_pieces(p) if ws == 1 else 1
+    if with_e2e and not (args.no_e2e or args.plain) and npieces > 1:
+        e2e = time_e2e_pipelined(li, p, inp, calls, dev, npieces, K, warmup, flush_l2)
+    elif with_e2e and not (args.no_e2e or args.plain):
         # every device tensor a call reads is refreshed once per step (pieces
         # that share one, such as a paged pool, copy it once)
         hosts = []

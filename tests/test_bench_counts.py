@@ -88,3 +88,22 @@ def test_default_workload_is_the_largest_configuration():
         p, x = bench.make_workload(name)
         sizes[name] = bench.work_counts(p, x)["flops"]
     assert max(sizes, key=sizes.get) == bench.DEFAULT_WORKLOAD == "quant_varlen"
+
+
+def test_end_to_end_pieces_tile_the_rows():
+    """The overlapped end-to-end leg splits a problem into contiguous row
+    pieces (the multi-GPU row split); they must cover every row once."""
+    import numpy as np
+
+    from sparse_attention_top_n1_b200 import shard
+    for name, want in (("cfg2", 1), ("dsa_prefill", 2), ("quant_varlen", 7), ("paged_decode", 1)):
+        p, inp = bench.make_workload(name)
+        n = bench.e2e_pieces(p)
+        assert n == want, name
+        aq, ak, cr = inp.get("act_q"), inp.get("act_k"), inp.get("cmp_residual_k")
+        cost = shard.row_costs(p, aq, ak, cr)
+        seen = np.zeros(p.rows, dtype=np.int64)
+        for r0, r1 in shard.split_rows(cost, n):
+            for pc in shard.pieces_for_range(p, r0, r1, aq, ak, cr):
+                seen[pc.r0:pc.r1] += 1
+        assert np.all(seen == 1), name

@@ -845,6 +845,68 @@ def sfa_reference(args, rank):
     return 0
 
 
+def sfa_e2e_pipelined(li, p, inp, d, pr_whole, out, lse, status, npieces, steps, warmup, flush_l2):
+    """End to end with host buffers for a one-batch BSND problem, transfers
+    overlapped with the work: the query rows are split into `npieces`
+    contiguous pieces (one li_sparse_attention call each); one stream copies
+    the keys and values and then each piece's query and index rows in, one
+    runs the calls as their inputs land, one copies each piece's output rows
+    out.  The pieces' outputs are checked bit for bit against the whole call."""
+    import dataclasses
+
+    import torch
+    dev = out.device
+    ref_o, ref_l = out.clone(), lse.clone()
+    shared = [(inp[k].contiguous().pin_memory(), d[k]) for k in ("key", "value")]
+    bounds = [p.rows * j // npieces for j in range(npieces + 1)]
+    pieces = []
+    for r0, r1 in zip(bounds, bounds[1:]):
+        pr = li.make_sfa_params(dataclasses.replace(p, S1=r1 - r0))
+        q_d, i_d = d["query"][:, r0:r1], d["sparse_indices"][r0:r1]
+        copies = [(inp["query"][:, r0:r1].contiguous().pin_memory(), q_d),
+                  (inp["sparse_indices"][r0:r1].contiguous().pin_memory(), i_d)]
+        ho = torch.empty(out[r0:r1].shape, dtype=out.dtype).pin_memory()
+        pieces.append((pr, q_d, i_d, copies, out[r0:r1], lse[r0:r1], ho))
+    h2d = sum(h.numel() * h.element_size() for h, _ in shared)
+    h2d += sum(h.numel() * h.element_size() for pc in pieces for h, _ in pc[3])
+    d2h = out.numel() * out.element_size()
+    s_in, s_run, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    main = torch.cuda.current_stream(dev)
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    st, en = [mk() for _ in range(steps + warmup)], [mk() for _ in range(steps + warmup)]
+    for s_ in range(steps + warmup):
+        flush_l2()
+        st[s_].record(main)
+        for x in (s_in, s_run, s_out):
+            x.wait_stream(main)
+        with torch.cuda.stream(s_in):
+            for h, dv in shared:
+                dv.copy_(h, non_blocking=True)
+        for pr, q_d, i_d, copies, o_d, l_d, ho in pieces:
+            with torch.cuda.stream(s_in):
+                for h, dv in copies:
+                    dv.copy_(h, non_blocking=True)
+            landed = s_in.record_event()
+            s_run.wait_event(landed)
+            with torch.cuda.stream(s_run):
+                li.li_sparse_attention(pr, q_d, d["key"], d["value"], i_d, None, None, None, o_d, l_d, status)
+            done = s_run.record_event()
+            s_out.wait_event(done)
+            with torch.cuda.stream(s_out):
+                ho.copy_(o_d, non_blocking=True)
+        main.wait_stream(s_out)
+        main.wait_stream(s_run)
+        en[s_].record(main)
+    torch.cuda.synchronize()
+    if not (torch.equal(out.view(torch.int16), ref_o.view(torch.int16))
+            and torch.equal(lse.view(torch.int32), ref_l.view(torch.int32))):
+        raise SystemExit("sparse attention end-to-end pieces differ from the whole call")
+    e_ms = allreduce_max(sum(st[s_].elapsed_time(en[s_]) for s_ in range(warmup, steps + warmup)))
+    return {"value": p.rows * steps / (e_ms * 1e-3), "unit": SFA_UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "pieces": len(pieces),
+            "overlap": "host->device copies, the calls and device->host copies on three streams, by row piece"}
+
+
 def sfa_main(args, ws, rank, local):
     """One step = one li_sparse_attention call over the whole workload; under
     torchrun every rank runs its own problem of the same shape (weak scaling)."""
@@ -909,7 +971,12 @@ def sfa_main(args, ws, rank, local):
     roof = {k: kern[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic", "peak_source")}
     roof["kernel"] = "sfa_kernel"
     e2e = None
-    if not (args.no_e2e or args.plain):
+    sfa_pieces = (min(8, p.rows // 2048) if (p.layout_q == "BSND" and p.B == 1 and "act_q" not in inp)
+                  else 1)
+    if not (args.no_e2e or args.plain) and sfa_pieces > 1:
+        e2e = sfa_e2e_pipelined(li, p, inp, d, pr, out, lse, status, sfa_pieces, K, args.warmup, flush_l2)
+        e2e["value"] *= ws
+    elif not (args.no_e2e or args.plain):
         host = {k: v.pin_memory() for k, v in inp.items()}
         hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         h2d = sum(v.numel() * v.element_size() for v in host.values())
